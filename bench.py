@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Throughput of the log-linear attention forward (Mamba-2 form) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--path auto|simt|tcgen05]
+
+One step is one forward over one batch of the workload (all of: decay scan,
+chunk states, Fenwick block merge, intra-chunk part, lam-weighted readout), with
+inputs resident in HBM.  Default workload: B=4, H=32, T=8192, d_k=d_v=64, bf16
+q/k/v, fp32 log_a/lam (L=14), fp32 out; synthetic seeded inputs.  The metric is
+tokens/s (tokens = sum of sequence lengths; heads are inside a token).  Under
+torchrun each rank runs its own batch (weak scaling, no collective on the data
+path); the time is the max over ranks.
+
+Prints ONE JSON line (rank 0) with the throughput, the dominant kernel's
+roofline fraction against the measured HBM bandwidth, the CPU oracle baseline,
+the end-to-end figure through the host-buffer C entry point, launch count and
+SM clocks sampled during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "log-linear attn fwd tokens/s at T=8K,H=32,d=64; % of roofline (1×B200)"
+DEFAULT_WORKLOAD = "t8k_d64_bf16"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------------
+# accounting
+# ---------------------------------------------------------------------------------------------
+def algorithmic_bytes(w, total_tokens):
+    """Bytes the method must move: read q, k, v, log_a, lam; write out (fp32)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    per = (2 * w.dk + w.dv) * esz + 4 * w.dv + 4 + 4 * w.L
+    return per * total_tokens * w.H, per
+
+
+def algorithmic_flops(w, lengths, chunk):
+    """Dense-tile FLOPs of the chunkwise form: intra 2C^2(dk+dv), chunk state 2C dk dv,
+    readout 2C dk dv per set bit of the chunk index."""
+    tot = 0
+    for n in lengths:
+        nch = (n + chunk - 1) // chunk
+        pc = sum(bin(c).count("1") for c in range(nch))
+        tot += nch * (2 * chunk * chunk * (w.dk + w.dv) + 2 * chunk * w.dk * w.dv) \
+            + pc * 2 * chunk * w.dk * w.dv
+    return tot * w.H
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_fenwick_state_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it matches these sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples = []
+        self.reasons = 0
+        self.err = None
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.err = f"nvml unavailable: {e}"
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(0.005)
+
+    def start(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                **({"error": self.err} if self.err else {})}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (the baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+def oracle_sample_rate(inp, heads, seconds_hint=None):
+    """Time the recurrent fp64 oracle on one sequence x `heads` heads; return (tok/s, desc, s)."""
+    import numpy as np
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:  # noqa: BLE001
+        threadpool_limits = None
+    start, n = inp.seq_slices()[0]
+    qf = inp.q.reshape(-1, inp.H, inp.dk)[start:start + n, :heads].transpose(1, 0, 2)
+    kf = inp.k.reshape(-1, inp.H, inp.dk)[start:start + n, :heads].transpose(1, 0, 2)
+    vf = inp.v.reshape(-1, inp.H, inp.dv)[start:start + n, :heads].transpose(1, 0, 2)
+    la = inp.log_a.reshape(-1, inp.H)[start:start + n, :heads].T
+    lm = inp.lam.reshape(-1, inp.H, inp.L)[start:start + n, :heads].transpose(1, 0, 2)
+    ctx = threadpool_limits(limits=1) if threadpool_limits else None
+    if ctx:
+        ctx.__enter__()
+    t0 = time.perf_counter()
+    O.llattn_recurrent_seq(np.ascontiguousarray(qf), np.ascontiguousarray(kf),
+                           np.ascontiguousarray(vf), np.ascontiguousarray(la),
+                           np.ascontiguousarray(lm))
+    dt = time.perf_counter() - t0
+    if ctx:
+        ctx.__exit__(None, None, None)
+    # tokens/s of the whole workload = (tokens of the sample * heads/H) / time
+    rate = n * (heads / inp.H) / dt
+    desc = (f"recurrent fp64 oracle form, 1 sequence x {heads} of {inp.H} heads x {n} tokens, "
+            f"{dt:.2f} s, numpy single thread")
+    return rate, desc, dt
+
+
+def run_reference(args, w, rank, world):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    from hierarchical_fenwick_state_b200 import inputs as I
+    if rank != 0:
+        return None
+    inp = I.make_inputs(w, seed=args.seed)
+    heads = 1
+    for _ in range(args.warmup):
+        oracle_sample_rate(inp, heads)
+    times, rates = [], []
+    for _ in range(args.steps):
+        r, desc, dt = oracle_sample_rate(inp, heads)
+        times.append(dt)
+        rates.append(r)
+    value = float(statistics.mean(rates))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": workload_config(w, None, None),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def workload_config(w, chunk, path):
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "L": w.L,
+           "inputs": f"{w.dtype} q/k/v, f32 log_a/lam, f32 out",
+           "log_a": f"-exp(N({w.log_a_mu},0.5))", "lam": "softplus(N(0,1))",
+           "l2": "inputs larger than L2 (no flush between steps)"}
+    if w.varlen:
+        cfg["varlen"] = f"{w.B} sequences, lengths U[{w.len_lo},{w.len_hi}]"
+    if chunk:
+        cfg["chunk"] = chunk
+    if path:
+        cfg["path"] = path
+    return cfg
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+def run_ours(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from hierarchical_fenwick_state_b200 import binding
+    from hierarchical_fenwick_state_b200 import inputs as I
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    inp = I.make_inputs(w, seed=args.seed + rank)
+    dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    q = torch.from_numpy(inp.q).to(dev).to(dt)
+    k = torch.from_numpy(inp.k).to(dev).to(dt)
+    v = torch.from_numpy(inp.v).to(dev).to(dt)
+    la = torch.from_numpy(inp.log_a).to(dev)
+    lm = torch.from_numpy(inp.lam).to(dev)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev) if inp.cu_seqlens is not None else None
+    out = torch.empty(inp.v.shape, dtype=torch.float32, device=dev)
+    lengths = [n for _, n in inp.seq_slices()]
+    total_tokens = int(sum(lengths))
+    path = args.path
+    # resolve the path and chunk the call will use
+    if path == "auto":
+        try:
+            binding.workspace_bytes(1 if dt == torch.bfloat16 else 0, "tcgen05", 0, inp.B, inp.H,
+                                    inp.T, inp.dk, inp.dv, cu is not None)
+            path = "tcgen05" if dt == torch.bfloat16 else "simt"
+        except binding.LLAttnError:
+            path = "simt"
+    chunk = 128 if path == "tcgen05" else (16 if inp.T <= 256 else 64)
+    nws = binding.workspace_bytes(1 if dt == torch.bfloat16 else 0, path, chunk, inp.B, inp.H,
+                                  inp.T, inp.dk, inp.dv, cu is not None)
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        binding.forward(q, k, v, la, lm, cu_seqlens=cu, T=inp.T, out=out, path=path, chunk=chunk,
+                        workspace=ws)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    binding.profile_read(reset=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    binding.profile(True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    binding.profile(False)
+    clk = clocks.stop()
+    ms_total = e0.elapsed_time(e1)
+    main_ms, main_n, launches = binding.profile_read(reset=True)
+    if dist:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    status = binding.device_status(clear=True)
+    if status:
+        raise RuntimeError(f"device status flags {status:#x} after the timed region")
+
+    ms_step = ms_total / args.steps
+    value = total_tokens * world / (ms_step / 1000.0)
+
+    # roofline of the dominant kernel
+    hbm_gbs, tflops, peak_kind = measured_peaks()
+    abytes, per_tok = algorithmic_bytes(w, total_tokens)
+    aflops = algorithmic_flops(w, lengths, chunk)
+    main_avg_s = (main_ms / main_n) / 1000.0 if main_n else ms_step / 1000.0
+    t_mem = abytes / (hbm_gbs * 1e9)
+    t_cmp = aflops / (tflops * 1e12)
+    kernel_key = f"{path}:{w.name}"
+    if t_mem >= t_cmp:
+        roof = {"bound": "hbm", "achieved": abytes / main_avg_s / 1e9, "peak": hbm_gbs,
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": aflops / main_avg_s / 1e12, "peak": tflops,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(kernel_key)
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "profiling-recipe fallback"
+    roof["kernel"] = kernel_key
+    roof["algorithmic_bytes_per_launch"] = abytes
+    roof["bytes_per_token_head"] = per_tok
+    roof["main_kernel_ms"] = main_avg_s * 1000.0
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": workload_config(w, chunk, path), "roofline": roof,
+        "gpu_launches": launches, "clocks": clk,
+    }
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    if not args.no_e2e:
+        in_dtype = 1 if inp.dtype == "bf16" else 0
+        if inp.dtype == "bf16":
+            hq = torch.from_numpy(I.bf16_bits(inp.q).view(np.int16)).pin_memory()
+            hk = torch.from_numpy(I.bf16_bits(inp.k).view(np.int16)).pin_memory()
+            hv = torch.from_numpy(I.bf16_bits(inp.v).view(np.int16)).pin_memory()
+        else:
+            hq = torch.from_numpy(inp.q).pin_memory()
+            hk = torch.from_numpy(inp.k).pin_memory()
+            hv = torch.from_numpy(inp.v).pin_memory()
+        hla = torch.from_numpy(inp.log_a).pin_memory()
+        hlm = torch.from_numpy(inp.lam).pin_memory()
+        hout = torch.empty(inp.v.shape, dtype=torch.float32).pin_memory()
+        hcu = torch.from_numpy(inp.cu_seqlens) if inp.cu_seqlens is not None else None
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hlm))
+        h2d += hcu.numel() * 4 if hcu is not None else 0
+        d2h = hout.numel() * 4
+
+        def e2e_step():
+            binding.fwd_host(in_dtype, hq, hk, hv, hla, hlm, hout, inp.B, inp.H, inp.T, inp.dk,
+                             inp.dv, cu_seqlens=hcu, stream=stream)
+
+        for _ in range(2):
+            e2e_step()
+        n_e2e = max(3, min(args.steps, 20))
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n_e2e):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2e_s = (time.perf_counter() - t0) / n_e2e
+        if dist:
+            t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_s = float(t.item())
+        ref_host = hout.numpy()
+        if not np.isfinite(ref_host).all():
+            raise RuntimeError("non-finite output through the host entry point")
+        line["e2e"] = {"value": total_tokens * world / e2e_s, "unit": "tokens/s",
+                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                       "steps": n_e2e, "entry": "llattn_fwd_host (pinned host buffers)"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, _ = oracle_sample_rate(inp, heads=min(inp.H, 12))
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": desc}
+    return line
+
+
+def main():
+    args = parse()
+    from hierarchical_fenwick_state_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

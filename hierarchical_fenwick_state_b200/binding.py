@@ -1,0 +1,204 @@
+"""Thin Python binding of the C ABI in include/llattn.h (argument marshalling only).
+
+Every step of the forward runs in libllattn.so's CUDA kernels; this module
+only checks tensors, passes raw device pointers, sizes and the current CUDA
+stream, and turns status codes into exceptions.  There is no CPU fallback:
+if the library is missing, ``lib()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libllattn.so")
+
+F32, BF16 = 0, 1
+PATHS = {"auto": 0, "simt": 1, "tcgen05": 2}
+
+# Every symbol include/llattn.h declares.
+EXPORTS = (
+    "llattn_abi_version", "llattn_status_str", "llattn_num_levels", "llattn_fwd",
+    "llattn_fwd_f32", "llattn_workspace_bytes", "llattn_fwd_ex", "llattn_device_status",
+    "llattn_last_cuda_error", "llattn_fwd_host", "llattn_profile", "llattn_profile_read",
+)
+
+_lib = None
+
+
+class LLAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().llattn_status_str(status).decode()
+        if status == 5:
+            msg += f" (cudaError {lib().llattn_last_cuda_error()})"
+        super().__init__(f"{where}: {msg} [status {status}]")
+
+
+def lib():
+    """Load libllattn.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m hierarchical_fenwick_state_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f_p, i_p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+    L.llattn_abi_version.restype = i
+    L.llattn_status_str.restype = ctypes.c_char_p
+    L.llattn_status_str.argtypes = [i]
+    L.llattn_num_levels.restype = i
+    L.llattn_num_levels.argtypes = [i]
+    L.llattn_fwd.restype = i
+    L.llattn_fwd.argtypes = [vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_fwd_f32.restype = i
+    L.llattn_fwd_f32.argtypes = [vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_workspace_bytes.restype = i
+    L.llattn_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+    L.llattn_fwd_ex.restype = i
+    L.llattn_fwd_ex.argtypes = [i, i, i, vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp,
+                                ctypes.c_size_t, vp]
+    L.llattn_device_status.restype = i
+    L.llattn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+    L.llattn_last_cuda_error.restype = i
+    L.llattn_fwd_host.restype = i
+    L.llattn_fwd_host.argtypes = [i, vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_profile.restype = i
+    L.llattn_profile.argtypes = [i]
+    L.llattn_profile_read.restype = i
+    L.llattn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                      ctypes.POINTER(ctypes.c_longlong),
+                                      ctypes.POINTER(ctypes.c_longlong), i]
+    _lib = L
+    return L
+
+
+def num_levels(T: int) -> int:
+    return int(lib().llattn_num_levels(int(T)))
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise LLAttnError(st, where)
+
+
+def workspace_bytes(in_dtype: int, path: str, chunk: int, B: int, H: int, T: int, dk: int,
+                    dv: int, varlen: bool) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().llattn_workspace_bytes(in_dtype, PATHS[path], chunk, B, H, T, dk, dv,
+                                        int(varlen), ctypes.byref(n)), "llattn_workspace_bytes")
+    return int(n.value)
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def forward(q, k, v, log_a, lam, *, cu_seqlens=None, T: Optional[int] = None, out=None,
+            path: str = "auto", chunk: int = 0, workspace=None, stream=None):
+    """o = llattn forward on device tensors (torch).  Returns out (fp32).
+
+    Dense: q,k [B,T,H,dk], v [B,T,H,dv], log_a [B,T,H], lam [B,T,H,L].
+    Packed: q,k [total,H,dk] ..., cu_seqlens int32 [B+1] on the device, and T
+    the bound on every sequence length.
+    """
+    import torch
+    dtype = q.dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q/k/v must be bf16 or fp32")
+    for t in (q, k, v, log_a, lam):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if k.dtype != dtype or v.dtype != dtype:
+        raise TypeError("q, k, v must share a dtype")
+    if log_a.dtype != torch.float32 or lam.dtype != torch.float32:
+        raise TypeError("log_a and lam must be fp32")
+    if cu_seqlens is None:
+        B, Tq, H, dk = q.shape
+        T = Tq
+    else:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+            raise TypeError("cu_seqlens must be an int32 CUDA tensor")
+        B = cu_seqlens.numel() - 1
+        _, H, dk = q.shape
+        if T is None:
+            raise ValueError("varlen needs T (max sequence length bound)")
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty(v.shape, dtype=torch.float32, device=v.device)
+    ws_ptr, ws_n = None, 0
+    if workspace is not None:
+        ws_ptr, ws_n = ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+    in_dtype = BF16 if dtype == torch.bfloat16 else F32
+    cu_ptr = ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None
+    st = lib().llattn_fwd_ex(in_dtype, PATHS[path], int(chunk), ctypes.c_void_p(q.data_ptr()),
+                             ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+                             ctypes.c_void_p(log_a.data_ptr()), ctypes.c_void_p(lam.data_ptr()),
+                             ctypes.c_void_p(out.data_ptr()), int(B), int(H), int(T), int(dk),
+                             int(dv), cu_ptr, ws_ptr, ws_n, _stream_handle(stream))
+    _check(st, "llattn_fwd_ex")
+    return out
+
+
+def fwd(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None, stream=None):
+    """Direct call of llattn_fwd (bf16 inputs, default path) on raw tensors."""
+    st = lib().llattn_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                          ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(log_a.data_ptr()),
+                          ctypes.c_void_p(lam.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                          int(B), int(H), int(T), int(dk), int(dv),
+                          ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None,
+                          _stream_handle(stream))
+    _check(st, "llattn_fwd")
+    return out
+
+
+def fwd_f32(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None, stream=None):
+    st = lib().llattn_fwd_f32(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                              ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(log_a.data_ptr()),
+                              ctypes.c_void_p(lam.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                              int(B), int(H), int(T), int(dk), int(dv),
+                              ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None,
+                              _stream_handle(stream))
+    _check(st, "llattn_fwd_f32")
+    return out
+
+
+def fwd_host(in_dtype: int, q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None,
+             stream=None):
+    """llattn_fwd_host on host buffers (numpy arrays or pinned CPU tensors; q/k/v as
+    uint16 bf16 bit patterns for in_dtype=BF16).  Copies in, computes, copies out."""
+    def ptr(x):
+        if x is None:
+            return None
+        if hasattr(x, "data_ptr"):
+            return ctypes.c_void_p(x.data_ptr())
+        return ctypes.c_void_p(x.ctypes.data)
+    st = lib().llattn_fwd_host(in_dtype, ptr(q), ptr(k), ptr(v), ptr(log_a), ptr(lam), ptr(out),
+                               int(B), int(H), int(T), int(dk), int(dv), ptr(cu_seqlens),
+                               _stream_handle(stream) if stream is not None else None)
+    _check(st, "llattn_fwd_host")
+    return out
+
+
+def profile(enable: bool):
+    _check(lib().llattn_profile(int(enable)), "llattn_profile")
+
+
+def profile_read(reset: bool = True):
+    """(main-kernel device ms summed, main-kernel launches timed, total kernel launches)."""
+    ms, n, tot = ctypes.c_double(0), ctypes.c_longlong(0), ctypes.c_longlong(0)
+    _check(lib().llattn_profile_read(ctypes.byref(ms), ctypes.byref(n), ctypes.byref(tot),
+                                     int(reset)), "llattn_profile_read")
+    return float(ms.value), int(n.value), int(tot.value)
+
+
+def device_status(clear: bool = True) -> int:
+    flags = ctypes.c_uint(0)
+    st = lib().llattn_device_status(ctypes.byref(flags), int(clear))
+    if st not in (0, 6):
+        _check(st, "llattn_device_status")
+    return int(flags.value)

@@ -1,0 +1,393 @@
+// Host side of the C ABI declared in include/llattn.h: argument validation,
+// workspace management, path dispatch and the device status word.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+#include <vector>
+
+#include "../../include/llattn.h"
+#include "llattn_internal.h"
+
+// Per-device status word: kernels OR LLATTN_DEV_* bits into it.
+__device__ unsigned int g_llattn_status;
+
+namespace {
+
+thread_local int t_last_cuda = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  unsigned int* status = nullptr;
+  void* stage = nullptr;  // llattn_fwd_host staging (inputs, output, cu_seqlens)
+  size_t stage_bytes = 0;
+};
+
+std::mutex g_mu;
+std::mutex g_host_mu;
+DeviceState g_dev[kMaxDevices];
+
+llattn_status cuda_fail(cudaError_t e) {
+  t_last_cuda = static_cast<int>(e);
+  return LLATTN_ERR_CUDA;
+}
+
+size_t round_up_host(size_t x) { return (x + 255) / 256 * 256; }
+
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int default_chunk(int path, int T) {
+  if (path == LLATTN_PATH_TCGEN05) return 128;
+  return T <= 256 ? 16 : 64;
+}
+
+// Resolve AUTO, the chunk length, and check that the chosen path takes the shape.
+llattn_status resolve(int in_dtype, int* path, int* chunk, int T, int dk, int dv) {
+  if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+  if (*path < LLATTN_PATH_AUTO || *path > LLATTN_PATH_TCGEN05) return LLATTN_ERR_ARG;
+  if (*path == LLATTN_PATH_AUTO) {
+    const int c = *chunk ? *chunk : default_chunk(LLATTN_PATH_TCGEN05, T);
+    *path = (in_dtype == LLATTN_BF16 && llattn::tc_supports(in_dtype, dk, dv, c))
+                ? LLATTN_PATH_TCGEN05 : LLATTN_PATH_SIMT;
+  }
+  if (*chunk == 0) *chunk = default_chunk(*path, T);
+  if (!pow2(*chunk)) return LLATTN_ERR_ARG;
+  if (*path == LLATTN_PATH_SIMT) {
+    if (*chunk < 8 || *chunk > 64) return LLATTN_ERR_ARG;
+  } else {
+    if (in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+    if (!llattn::tc_supports(in_dtype, dk, dv, *chunk)) return LLATTN_ERR_UNSUPPORTED;
+  }
+  return LLATTN_OK;
+}
+
+size_t workspace_for(int path, int chunk, int nseq, int H, int T, int dk, int dv) {
+  if (path == LLATTN_PATH_SIMT) return llattn::simt_workspace_bytes(nseq, H, T, dk, dv, chunk);
+  return llattn::tc_workspace_bytes(nseq, H, T, dk, dv, chunk);
+}
+
+llattn_status device_state(DeviceState** out, int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return LLATTN_ERR_ARG;
+  DeviceState& d = g_dev[dev];
+  if (d.status == nullptr) {
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_llattn_status);
+    if (e != cudaSuccess) {
+      d.status = nullptr;
+      return cuda_fail(e);
+    }
+  }
+  *out = &d;
+  *dev_out = dev;
+  return LLATTN_OK;
+}
+
+llattn_status forward(int in_dtype, int path, int chunk, const void* q, const void* k,
+                      const void* v, const float* log_a, const float* lam, float* out, int B,
+                      int H, int T, int dk, int dv, const int* cu_seqlens, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || T < 0) return LLATTN_ERR_SHAPE;
+  if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
+  if (T > (1 << 24) || H > 65535 || B > 65535) return LLATTN_ERR_SHAPE;
+  llattn_status s = resolve(in_dtype, &path, &chunk, T, dk, dv);
+  if (s != LLATTN_OK) return s;
+  if (B == 0 || H == 0 || T == 0) return LLATTN_OK;  // nothing to compute
+  if (!q || !k || !v || !log_a || !lam || !out) return LLATTN_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(log_a, 4) || !aligned(lam, 4) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return LLATTN_ERR_ALIGN;
+  const void* ins[5] = {q, k, v, log_a, lam};
+  for (const void* p : ins)
+    if (p == static_cast<const void*>(out)) return LLATTN_ERR_ARG;
+  const int L = llattn_num_levels(T);
+  if (cu_seqlens == nullptr) {
+    // dense: the whole output range must not overlap any input range
+    const unsigned long long ntok = (unsigned long long)B * T;
+    if (ntok * H * (unsigned long long)(dk > dv ? dk : dv) > (1ull << 40)) return LLATTN_ERR_SHAPE;
+    const size_t esz = in_dtype == LLATTN_BF16 ? 2 : 4;
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out);
+    const uintptr_t o1 = o0 + ntok * H * dv * sizeof(float);
+    const struct { const void* p; size_t n; } rng[5] = {
+        {q, ntok * H * dk * esz}, {k, ntok * H * dk * esz}, {v, ntok * H * dv * esz},
+        {log_a, ntok * H * sizeof(float)}, {lam, ntok * H * L * sizeof(float)}};
+    for (const auto& r : rng) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(r.p), a1 = a0 + r.n;
+      if (a0 < o1 && o0 < a1) return LLATTN_ERR_ARG;
+    }
+  }
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  if ((s = device_state(&ds, &dev)) != LLATTN_OK) return s;
+  const size_t need = workspace_for(path, chunk, B, H, T, dk, dv);
+  void* ws = workspace;
+  std::unique_lock<std::mutex> lock(g_mu, std::defer_lock);
+  if (workspace != nullptr) {
+    if (workspace_bytes < need || !aligned(workspace, 256)) return LLATTN_ERR_WORKSPACE;
+  } else if (need > 0) {
+    lock.lock();
+    if (ds->ws_bytes < need) {
+      cudaError_t e;
+      if (ds->ws) {
+        if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
+        cudaFree(ds->ws);
+        ds->ws = nullptr;
+        ds->ws_bytes = 0;
+      }
+      if ((e = cudaMalloc(&ds->ws, need)) != cudaSuccess) {
+        ds->ws = nullptr;
+        return cuda_fail(e);
+      }
+      ds->ws_bytes = need;
+    }
+    ws = ds->ws;
+  }
+  llattn::Problem p{in_dtype, q, k, v, log_a, lam, out, B, H, T, dk, dv, L, cu_seqlens,
+                    ds->status};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = path == LLATTN_PATH_SIMT ? llattn::simt_forward(p, chunk, ws, st)
+                                           : llattn::tc_forward(p, chunk, ws, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return LLATTN_OK;
+}
+
+// ---- launch accounting ----
+std::atomic<long long> g_total_launches{0};
+std::atomic<bool> g_profiling{false};
+std::mutex g_prof_mu;
+struct EvPair { cudaEvent_t a, b; };
+std::vector<EvPair> g_prof_events;   // recorded pairs not yet read
+std::vector<cudaEvent_t> g_event_pool;
+thread_local cudaEvent_t t_open_event = nullptr;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+}  // namespace
+
+namespace llattn {
+
+void count_launch(int n) { g_total_launches.fetch_add(n); }
+
+void main_kernel_begin(cudaStream_t st) {
+  if (!g_profiling.load()) return;
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  t_open_event = pool_event();
+  if (t_open_event) cudaEventRecord(t_open_event, st);
+}
+
+void main_kernel_end(cudaStream_t st) {
+  if (!g_profiling.load() || t_open_event == nullptr) return;
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  cudaEvent_t b = pool_event();
+  if (b == nullptr) return;
+  cudaEventRecord(b, st);
+  g_prof_events.push_back({t_open_event, b});
+  t_open_event = nullptr;
+}
+
+}  // namespace llattn
+
+extern "C" {
+
+llattn_status llattn_profile(int enable) {
+  g_profiling.store(enable != 0);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_profile_read(double* main_kernel_ms, long long* main_launches,
+                                  long long* total_launches, int reset) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  double ms = 0.0;
+  for (const EvPair& p : g_prof_events) {
+    cudaError_t e = cudaEventSynchronize(p.b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    float x = 0.f;
+    if ((e = cudaEventElapsedTime(&x, p.a, p.b)) != cudaSuccess) return cuda_fail(e);
+    ms += x;
+  }
+  if (main_kernel_ms) *main_kernel_ms = ms;
+  if (main_launches) *main_launches = (long long)g_prof_events.size();
+  if (total_launches) *total_launches = g_total_launches.load();
+  if (reset) {
+    for (const EvPair& p : g_prof_events) {
+      g_event_pool.push_back(p.a);
+      g_event_pool.push_back(p.b);
+    }
+    g_prof_events.clear();
+    g_total_launches.store(0);
+  }
+  return LLATTN_OK;
+}
+
+
+int llattn_abi_version(void) { return 1; }
+
+const char* llattn_status_str(llattn_status s) {
+  switch (s) {
+    case LLATTN_OK: return "ok";
+    case LLATTN_ERR_ARG: return "invalid argument";
+    case LLATTN_ERR_SHAPE: return "unsupported or out-of-range shape";
+    case LLATTN_ERR_ALIGN: return "misaligned pointer";
+    case LLATTN_ERR_DTYPE: return "unsupported dtype";
+    case LLATTN_ERR_CUDA: return "CUDA error";
+    case LLATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    case LLATTN_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case LLATTN_ERR_UNSUPPORTED: return "no kernel for this configuration";
+  }
+  return "unknown status";
+}
+
+int llattn_num_levels(int T) {
+  if (T <= 1) return 1;
+  int bits = 0;
+  unsigned x = static_cast<unsigned>(T - 1);
+  while (x) { ++bits; x >>= 1; }
+  return 1 + bits;
+}
+
+llattn_status llattn_workspace_bytes(int in_dtype, int path, int chunk, int B, int H, int T,
+                                     int dk, int dv, int varlen, size_t* bytes) {
+  (void)varlen;  // dense and packed batches are sized alike (T bounds every sequence)
+  if (!bytes) return LLATTN_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || T > (1 << 24)) return LLATTN_ERR_SHAPE;
+  if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
+  llattn_status s = resolve(in_dtype, &path, &chunk, T, dk, dv);
+  if (s != LLATTN_OK) return s;
+  *bytes = (B == 0 || H == 0 || T == 0) ? 0 : workspace_for(path, chunk, B, H, T, dk, dv);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_fwd(const void* q, const void* k, const void* v, const float* log_a,
+                         const float* lam, float* out, int B, int H, int T, int dk, int dv,
+                         const int* cu_seqlens, void* stream) {
+  return forward(LLATTN_BF16, LLATTN_PATH_AUTO, 0, q, k, v, log_a, lam, out, B, H, T, dk, dv,
+                 cu_seqlens, nullptr, 0, stream);
+}
+
+llattn_status llattn_fwd_f32(const float* q, const float* k, const float* v, const float* log_a,
+                             const float* lam, float* out, int B, int H, int T, int dk, int dv,
+                             const int* cu_seqlens, void* stream) {
+  return forward(LLATTN_F32, LLATTN_PATH_SIMT, 0, q, k, v, log_a, lam, out, B, H, T, dk, dv,
+                 cu_seqlens, nullptr, 0, stream);
+}
+
+llattn_status llattn_fwd_ex(int in_dtype, int path, int chunk, const void* q, const void* k,
+                            const void* v, const float* log_a, const float* lam, float* out,
+                            int B, int H, int T, int dk, int dv, const int* cu_seqlens,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return forward(in_dtype, path, chunk, q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens,
+                 workspace, workspace_bytes, stream);
+}
+
+llattn_status llattn_device_status(unsigned int* flags, int clear) {
+  if (!flags) return LLATTN_ERR_ARG;
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  llattn_status s = device_state(&ds, &dev);
+  if (s != LLATTN_OK) return s;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned int v = 0;
+  if ((e = cudaMemcpy(&v, ds->status, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e);
+  if (clear && v) {
+    if ((e = cudaMemset(ds->status, 0, sizeof(v))) != cudaSuccess) return cuda_fail(e);
+  }
+  *flags = v;
+  return (v & LLATTN_DEV_WAIT_TIMEOUT) ? LLATTN_ERR_TIMEOUT : LLATTN_OK;
+}
+
+llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const void* v,
+                              const float* log_a, const float* lam, float* out, int B, int H,
+                              int T, int dk, int dv, const int* cu_seqlens, void* stream) {
+  if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+  if (B < 0 || H < 0 || T < 0 || T > (1 << 24)) return LLATTN_ERR_SHAPE;
+  if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
+  if (B == 0 || H == 0 || T == 0) return LLATTN_OK;
+  if (!q || !k || !v || !log_a || !lam || !out) return LLATTN_ERR_ARG;
+  long long total = (long long)B * T;
+  if (cu_seqlens) {
+    if (cu_seqlens[0] != 0) return LLATTN_ERR_ARG;
+    for (int i = 0; i < B; ++i) {
+      const int len = cu_seqlens[i + 1] - cu_seqlens[i];
+      if (len < 0 || len > T) return LLATTN_ERR_SHAPE;
+    }
+    total = cu_seqlens[B];
+  }
+  if (total * H * (long long)(dk > dv ? dk : dv) > (1ll << 40)) return LLATTN_ERR_SHAPE;
+  const int L = llattn_num_levels(T);
+  const size_t esz = in_dtype == LLATTN_BF16 ? 2 : 4;
+  const size_t nq = round_up_host((size_t)total * H * dk * esz);
+  const size_t nv = round_up_host((size_t)total * H * dv * esz);
+  const size_t na = round_up_host((size_t)total * H * sizeof(float));
+  const size_t nl = round_up_host((size_t)total * H * L * sizeof(float));
+  const size_t no = round_up_host((size_t)total * H * dv * sizeof(float));
+  const size_t nc = round_up_host((size_t)(B + 1) * sizeof(int));
+  const size_t need = 2 * nq + nv + na + nl + no + nc;
+  std::lock_guard<std::mutex> hold(g_host_mu);
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  llattn_status s = device_state(&ds, &dev);
+  if (s != LLATTN_OK) return s;
+  cudaError_t e;
+  if (ds->stage_bytes < need) {
+    if (ds->stage) {
+      if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
+      cudaFree(ds->stage);
+      ds->stage = nullptr;
+      ds->stage_bytes = 0;
+    }
+    if ((e = cudaMalloc(&ds->stage, need)) != cudaSuccess) {
+      ds->stage = nullptr;
+      return cuda_fail(e);
+    }
+    ds->stage_bytes = need;
+  }
+  char* b = static_cast<char*>(ds->stage);
+  char* dq = b; b += nq;
+  char* dk_ = b; b += nq;
+  char* dv_ = b; b += nv;
+  float* da = reinterpret_cast<float*>(b); b += na;
+  float* dl = reinterpret_cast<float*>(b); b += nl;
+  float* dout = reinterpret_cast<float*>(b); b += no;
+  int* dcu = cu_seqlens ? reinterpret_cast<int*>(b) : nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const struct { void* d; const void* h; size_t n; } cp[6] = {
+      {dq, q, (size_t)total * H * dk * esz}, {dk_, k, (size_t)total * H * dk * esz},
+      {dv_, v, (size_t)total * H * dv * esz}, {da, log_a, (size_t)total * H * sizeof(float)},
+      {dl, lam, (size_t)total * H * L * sizeof(float)},
+      {dcu, cu_seqlens, (size_t)(B + 1) * sizeof(int)}};
+  for (const auto& c : cp) {
+    if (c.d == nullptr || c.n == 0) continue;
+    if ((e = cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+      return cuda_fail(e);
+  }
+  s = forward(in_dtype, LLATTN_PATH_AUTO, 0, dq, dk_, dv_, da, dl, dout, B, H, T, dk, dv, dcu,
+              nullptr, 0, stream);
+  if (s != LLATTN_OK) return s;
+  if ((e = cudaMemcpyAsync(out, dout, (size_t)total * H * dv * sizeof(float),
+                           cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e);
+  return LLATTN_OK;
+}
+
+int llattn_last_cuda_error(void) { return t_last_cuda; }
+
+}  // extern "C"

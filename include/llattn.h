@@ -1,0 +1,185 @@
+/*
+ * llattn.h - C ABI of the B200-native log-linear attention forward (Mamba-2 form).
+ *
+ * Operation.  For every sequence, head and 0-based sequence-local position t:
+ *
+ *   o_t = sum_{s <= t} lam[t, l(t,s)] * (prod_{r=s+1..t} a_r) * (q_t . k_s) * v_s
+ *   l(t,s) = 0 if s == t, else 1 + floor(log2(t XOR s)),   a_r = exp(log_a[r]),
+ *
+ * i.e. linear attention whose causal mask is replaced by the hierarchical
+ * (HODLR) mask of a Fenwick-tree partition of the prefix, with Mamba-2's
+ * scalar selective gate and one weight per (query token, level).  Sources:
+ * "Log-Linear Attention" (gist.science summaries, Italian "Sommario tecnico"
+ * section 2 and Spanish "Resumen tecnico" section 2): the Fenwick partition into
+ * buckets of exponentially growing size (Partizionamento Gerarchico / Particion
+ * Jerarquica), the hierarchical mask M_H (Matrici Gerarchiche), the O(log T)
+ * level states combined with per-level weights (Forma Ricorrente), the
+ * chunkwise-parallel forward in O(T log T) (Training bullet / Algoritmo de
+ * Entrenamiento), and the Log-Linear Mamba-2 variant (Variantes Propuestas 1).
+ * lam is applied as given (the caller applies any positivity transform); there
+ * is no softmax, no 1/sqrt(d) scale and no normalisation.
+ *
+ * Layouts (all row-major, contiguous, token-major, level innermost):
+ *   q, k   [B, T, H, dk]        v [B, T, H, dv]       out [B, T, H, dv] (fp32)
+ *   log_a  [B, T, H] (fp32)     lam [B, T, H, L] (fp32), L = llattn_num_levels(T)
+ * Packed variable-length batches (cu_seqlens != NULL): B = number of sequences,
+ * tensors are [total, H, .] with total = cu_seqlens[B], cu_seqlens is a DEVICE
+ * int32 array of B+1 non-decreasing offsets starting at 0, and T is an upper
+ * bound on every sequence length (it fixes L and the launch grid).  Fenwick
+ * positions and the gate product restart at every sequence start.
+ *
+ * Ownership.  Every tensor pointer is caller-owned DEVICE memory; the library
+ * never frees or retains it.  q, k, v and out must be 16-byte aligned, log_a and
+ * lam 4-byte aligned; out must not alias any input.  Calls are asynchronous on
+ * `stream` (a cudaStream_t; NULL = legacy default stream) and return once the
+ * kernels are enqueued; `out` is fully overwritten for every token of every
+ * sequence (rows outside [0, total) are not touched).
+ *
+ * Output precision.  out is fp32 for every input type: rounding the output to
+ * bf16 alone moves it by up to ~4% of its RMS on these heavy-tailed outputs.
+ *
+ * Errors.  Every entry point returns an llattn_status and never aborts.  Bad
+ * arguments are rejected before any launch.  Launch failures map to
+ * LLATTN_ERR_CUDA.  Conditions only the device can see (a varlen sequence longer
+ * than T, a bounded wait that ran out) set bits in a per-device status word that
+ * llattn_device_status() reads; the affected output rows are then unspecified.
+ */
+#ifndef LLATTN_H_
+#define LLATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLATTN_API __attribute__((visibility("default")))
+#else
+#define LLATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LLATTN_OK = 0,
+  LLATTN_ERR_ARG = 1,         /* null pointer, negative size, aliasing */
+  LLATTN_ERR_SHAPE = 2,       /* unsupported dk/dv, T or sizes out of range */
+  LLATTN_ERR_ALIGN = 3,       /* pointer misaligned (16 B for q/k/v/out, 4 B for log_a/lam) */
+  LLATTN_ERR_DTYPE = 4,       /* unknown input dtype code */
+  LLATTN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  LLATTN_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out (see llattn_device_status) */
+  LLATTN_ERR_WORKSPACE = 7,   /* caller workspace too small or misaligned */
+  LLATTN_ERR_UNSUPPORTED = 8  /* valid request this build has no kernel for */
+} llattn_status;
+
+/* Input element types for llattn_fwd_ex. */
+enum { LLATTN_F32 = 0, LLATTN_BF16 = 1 };
+
+/* Kernel paths for llattn_fwd_ex.
+ *   AUTO     tcgen05 path where one exists for the shape, else SIMT.
+ *   SIMT     CUDA-core kernels (any dk, dv in {32,64,128}; fp32 or bf16 inputs).
+ *   TCGEN05  tensor-core kernels (bf16 inputs only). */
+enum { LLATTN_PATH_AUTO = 0, LLATTN_PATH_SIMT = 1, LLATTN_PATH_TCGEN05 = 2 };
+
+/* Device status bits (llattn_device_status). */
+enum {
+  LLATTN_DEV_SEQ_TOO_LONG = 1u,  /* a varlen sequence was longer than T */
+  LLATTN_DEV_WAIT_TIMEOUT = 2u,  /* an mbarrier / pipeline wait hit its iteration limit */
+  LLATTN_DEV_BAD_CU_SEQLENS = 4u /* cu_seqlens decreasing */
+};
+
+/* Version of this ABI (increments on any signature change). */
+LLATTN_API int llattn_abi_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+LLATTN_API const char* llattn_status_str(llattn_status s);
+
+/* Number of Fenwick levels for sequences of at most T tokens: 1 + ceil(log2 T)
+ * (1 for T <= 1).  This is the innermost extent of lam. */
+LLATTN_API int llattn_num_levels(int T);
+
+/*
+ * llattn_fwd - forward with bf16 q, k, v (each a uint16 bf16 bit pattern),
+ * fp32 log_a and lam, fp32 out, on the default (tensor-core) path.  Scratch
+ * for inter-chunk states comes from a per-device buffer the library grows on
+ * demand and keeps until exit; calls that overlap on the GPU (two streams)
+ * must use llattn_fwd_ex with their own workspaces instead.
+ * B, H >= 0, T >= 0, dk and dv in {32, 64, 128}.  Returns LLATTN_OK on success.
+ */
+LLATTN_API llattn_status llattn_fwd(const void* q, const void* k, const void* v, const float* log_a,
+                         const float* lam, float* out, int B, int H, int T, int dk, int dv,
+                         const int* cu_seqlens, void* stream);
+
+/* llattn_fwd_f32 - the same operation on fp32 q, k, v (CUDA-core fp32 path, no
+ * tensor cores, so results meet a 1e-4 relative bound).  Arguments as llattn_fwd. */
+LLATTN_API llattn_status llattn_fwd_f32(const float* q, const float* k, const float* v, const float* log_a,
+                             const float* lam, float* out, int B, int H, int T, int dk, int dv,
+                             const int* cu_seqlens, void* stream);
+
+/*
+ * llattn_workspace_bytes - device scratch that llattn_fwd_ex needs for this
+ * shape, dtype and path (0 is possible).  chunk = 0 selects the default chunk
+ * length of the path.  varlen != 0 sizes for packed sequences bounded by T.
+ */
+LLATTN_API llattn_status llattn_workspace_bytes(int in_dtype, int path, int chunk, int B, int H, int T,
+                                     int dk, int dv, int varlen, size_t* bytes);
+
+/*
+ * llattn_fwd_ex - the general entry point.
+ *   in_dtype   LLATTN_F32 or LLATTN_BF16 (type of q, k, v).
+ *   path       LLATTN_PATH_* (SIMT accepts both dtypes, TCGEN05 bf16 only).
+ *   chunk      chunk length (power of two; 0 = default of the path: SIMT 16 for
+ *              T <= 256 else 64, TCGEN05 128).  The result does not depend on it
+ *              beyond rounding.
+ *   workspace  caller-owned device scratch of at least llattn_workspace_bytes()
+ *              bytes (256-byte aligned), or NULL to use the library's per-device
+ *              buffer as llattn_fwd does.
+ */
+LLATTN_API llattn_status llattn_fwd_ex(int in_dtype, int path, int chunk, const void* q, const void* k,
+                            const void* v, const float* log_a, const float* lam, float* out,
+                            int B, int H, int T, int dk, int dv, const int* cu_seqlens,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * llattn_device_status - read (and, if clear != 0, reset) the status word of the
+ * current device.  Synchronises the device.  *flags receives LLATTN_DEV_* bits.
+ */
+LLATTN_API llattn_status llattn_device_status(unsigned int* flags, int clear);
+
+/*
+ * llattn_fwd_host - the forward on HOST buffers, for callers whose data is not
+ * on the GPU.  Copies q, k, v, log_a, lam (and cu_seqlens) into device staging
+ * memory the library owns (grown on demand, kept per device until exit), runs
+ * the default path (tensor cores for bf16, CUDA cores for fp32), copies out back
+ * and synchronises `stream` before returning.  Host buffers should be pinned
+ * (page-locked) for the copies to run at full speed.  in_dtype: LLATTN_BF16
+ * (q, k, v as uint16 bf16 bit patterns) or LLATTN_F32.  cu_seqlens, if not NULL,
+ * is a HOST int32 array [B+1]; the other arguments are as in llattn_fwd.
+ * Concurrent calls from several threads are serialised on an internal lock.
+ */
+LLATTN_API llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const void* v,
+                              const float* log_a, const float* lam, float* out, int B, int H,
+                              int T, int dk, int dv, const int* cu_seqlens, void* stream);
+
+/*
+ * Launch accounting, for benchmarks.  llattn_profile(1) starts recording a pair
+ * of CUDA events on the call's stream around the dominant kernel of every
+ * forward (the one that streams q, k, v, lam and writes out); llattn_profile(0)
+ * stops.  llattn_profile_read returns the summed device time of those kernels
+ * (synchronising on the recorded events), how many were timed, and how many
+ * kernels of this library were launched in total since the last reset (counted
+ * whether or not recording is on); reset != 0 clears all three.
+ */
+LLATTN_API llattn_status llattn_profile(int enable);
+LLATTN_API llattn_status llattn_profile_read(double* main_kernel_ms, long long* main_launches,
+                                             long long* total_launches, int reset);
+
+/* llattn_last_cuda_error - the cudaError_t behind the last LLATTN_ERR_CUDA of
+ * this thread (0 if none). */
+LLATTN_API int llattn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLATTN_H_ */

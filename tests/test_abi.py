@@ -1,0 +1,79 @@
+"""The C-ABI library loads, exports every declared symbol, and validates arguments (no GPU).
+
+Only entry points that return before touching CUDA are called here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hierarchical_fenwick_state_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "llattn.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"LLATTN_API\s+[\w\s\*]+?\b(llattn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_exports():
+    decl = declared_symbols()
+    assert "llattn_fwd" in decl and "llattn_fwd_f32" in decl
+    assert sorted(binding.EXPORTS) == decl
+
+
+def test_library_exports_every_declared_symbol():
+    lib = binding.lib()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_num_levels_and_strings():
+    lib = binding.lib()
+    assert [lib.llattn_num_levels(T) for T in (1, 2, 3, 256, 2048, 8192, 16384, 65536)] == \
+        [1, 2, 3, 9, 12, 14, 15, 17]
+    assert lib.llattn_abi_version() >= 1
+    for s in range(9):
+        assert lib.llattn_status_str(s)
+    assert lib.llattn_status_str(99) == b"unknown status"
+
+
+def _call_ex(**kw):
+    a = dict(in_dtype=1, path=0, chunk=0, q=0x1000, k=0x2000, v=0x3000, log_a=0x4000,
+             lam=0x5000, out=0x6000, B=1, H=1, T=16, dk=64, dv=64, cu=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return binding.lib().llattn_fwd_ex(a["in_dtype"], a["path"], a["chunk"], vp(a["q"]), vp(a["k"]),
+                                       vp(a["v"]), vp(a["log_a"]), vp(a["lam"]), vp(a["out"]),
+                                       a["B"], a["H"], a["T"], a["dk"], a["dv"],
+                                       vp(a["cu"]) if a["cu"] else None, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48), 2), (dict(dv=256), 2), (dict(T=-1), 2), (dict(B=-2), 2),
+    (dict(in_dtype=7), 4), (dict(path=9), 1), (dict(chunk=24, path=1), 1),
+    (dict(chunk=128, path=1), 1), (dict(in_dtype=0, path=2), 4),
+    (dict(q=0x1008), 3), (dict(out=0x6004), 3), (dict(lam=0x5002), 3),
+    (dict(q=0), 1), (dict(out=0x1000), 1),
+    # out overlaps lam's range (lam = 16 tokens * 5 levels * 4 B from 0x5000)
+    (dict(out=0x5010), 1),
+])
+def test_argument_errors_before_launch(kw, status):
+    assert _call_ex(**kw) == status
+
+
+def test_empty_problems_are_no_ops():
+    assert _call_ex(B=0) == 0
+    assert _call_ex(H=0) == 0
+    assert _call_ex(T=0) == 0
+
+
+def test_workspace_query():
+    n = binding.workspace_bytes(1, "simt", 64, 2, 4, 1000, 64, 64, False)
+    assert n > 0 and n % 256 == 0
+    assert binding.workspace_bytes(1, "simt", 64, 0, 4, 1000, 64, 64, False) == 0
+    with pytest.raises(binding.LLAttnError):
+        binding.workspace_bytes(1, "simt", 64, 1, 4, 1000, 48, 64, False)

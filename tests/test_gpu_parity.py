@@ -1,0 +1,154 @@
+"""GPU parity: the CUDA paths (through the C ABI) against the CPU fp64 oracle.
+
+Oracle-sized cases span several chunks and a ragged tail and compare every
+output element; full-size cases (the bench's launch configuration) compare
+sampled outputs the oracle computes one at a time.  Metric: max |gpu - oracle|
+divided by the RMS of the oracle output, <= 1e-4 for fp32 inputs and <= 2e-2 for
+bf16 inputs (fp32 accumulation, fp32 output).
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from hierarchical_fenwick_state_b200 import binding
+from hierarchical_fenwick_state_b200 import inputs as I
+
+from _llattn_cases import TOL, run
+
+pytestmark = pytest.mark.gpu
+
+W = I.WORKLOADS
+
+
+def _paths_for(inp):
+    paths = ["simt"]
+    if inp.dtype == "bf16":
+        try:
+            binding.workspace_bytes(1, "tcgen05", 0, inp.B, inp.H, inp.T, inp.dk, inp.dv,
+                                    inp.cu_seqlens is not None)
+            paths.append("tcgen05")
+        except binding.LLAttnError:
+            pass
+    return paths
+
+
+def _check(inp, ref, path, chunk=0):
+    got = run(inp, path=path, chunk=chunk)
+    assert np.isfinite(got).all(), "unwritten or non-finite outputs"
+    err = O.rel_max_err(got, ref)
+    assert err <= TOL[inp.dtype], f"{path} chunk={chunk}: rel max err {err:.3e}"
+    return err
+
+
+# ------------------------------------------------------------------------------------------------
+# Element-by-element parity on oracle-sized cases of each workload
+# ------------------------------------------------------------------------------------------------
+CASES = {
+    "t256_d32_f32": W["t256_d32_f32"],
+    "t256_d32_f32_ragged": I.shrink(W["t256_d32_f32"], T=250),
+    "t2k_d64_bf16": W["t2k_d64_bf16"],
+    "t8k_d64_bf16_h2": I.shrink(W["t8k_d64_bf16"], B=1, H=2),
+    "t8k_d64_bf16_ragged": I.shrink(W["t8k_d64_bf16"], B=2, H=1, T=8000),
+    "t64k_d128_bf16_t8k": I.shrink(W["t64k_d128_bf16"], H=2, T=8192),
+    "varlen_small": I.shrink(W["varlen8_d64_bf16"], H=2, T=3000, len_lo=1, len_hi=3000),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_parity_workloads(name):
+    inp = I.make_inputs(CASES[name], seed=0)
+    ref = O.llattn_recurrent(inp)
+    for path in _paths_for(inp):
+        _check(inp, ref, path)
+
+
+# ------------------------------------------------------------------------------------------------
+# Stress: decay regimes that reach the deep Fenwick levels, one level at a time
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", ["zero", "slow", "strong"])
+@pytest.mark.parametrize("base", ["t2k_d64_bf16", "t256_d32_f32"])
+def test_parity_decay_regimes(mode, base):
+    w = I.shrink(W[base], B=1, H=2) if base == "t2k_d64_bf16" else W[base]
+    inp = I.make_inputs(w, seed=1, log_a_mode=mode)
+    ref = O.llattn_recurrent(inp)
+    for path in _paths_for(inp):
+        _check(inp, ref, path)
+
+
+@pytest.mark.parametrize("level", [0, 1, 5, 6, 7, 8, 10, 11])
+def test_parity_one_hot_level(level):
+    w = I.shrink(W["t2k_d64_bf16"], B=1, H=2)
+    inp = I.make_inputs(w, seed=2, log_a_mode="zero", lam_mode="onehot", lam_level=level)
+    ref = O.llattn_recurrent(inp)
+    for path in _paths_for(inp):
+        _check(inp, ref, path)
+
+
+@pytest.mark.parametrize("chunk", [8, 16, 32, 64])
+def test_simt_chunk_invariance(chunk):
+    w = I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=1000)
+    inp = I.make_inputs(w, seed=3, log_a_mode="slow")
+    ref = O.llattn_recurrent(inp)
+    _check(inp, ref, "simt", chunk=chunk)
+
+
+# ------------------------------------------------------------------------------------------------
+# Edge cases
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 257])
+def test_edge_lengths(T):
+    for base in ("t2k_d64_bf16", "t256_d32_f32"):
+        w = I.shrink(W[base], B=2, H=1, T=T)
+        inp = I.make_inputs(w, seed=T)
+        ref = O.llattn_recurrent(inp)
+        for path in _paths_for(inp):
+            _check(inp, ref, path)
+
+
+def test_varlen_edge_lengths():
+    w = I.Workload("vl_edge", B=7, H=3, T=600, dk=64, dv=64, dtype="bf16", varlen=True)
+    inp = I.make_inputs(w, seed=5, lengths=np.array([0, 1, 129, 600, 64, 0, 2]))
+    ref = O.llattn_recurrent(inp)
+    for path in _paths_for(inp):
+        _check(inp, ref, path)
+
+
+def test_varlen_sequence_longer_than_bound_sets_status():
+    import torch
+    from _llattn_cases import to_device
+    w = I.Workload("vl_bad", B=2, H=1, T=64, dk=64, dv=64, dtype="bf16", varlen=True)
+    inp = I.make_inputs(w, seed=6, lengths=np.array([100, 10]))
+    t = to_device(inp)
+    out = torch.zeros(inp.v.shape, dtype=torch.float32, device="cuda:0")
+    binding.forward(t["q"], t["k"], t["v"], t["log_a"], t["lam"], cu_seqlens=t["cu"], T=64,
+                    out=out, path="simt")
+    torch.cuda.synchronize()
+    assert binding.device_status(clear=True) & 1
+
+
+def test_dims_32_and_128_mixed():
+    w = I.Workload("mixed", B=1, H=2, T=300, dk=32, dv=128, dtype="bf16")
+    inp = I.make_inputs(w, seed=8)
+    ref = O.llattn_recurrent(inp)
+    _check(inp, ref, "simt")
+
+
+# ------------------------------------------------------------------------------------------------
+# Full-size workloads in the bench's launch configuration: sampled outputs
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name", list(W))
+def test_full_size_sampled(name):
+    w = W[name]
+    inp = I.make_inputs(w, seed=0)
+    rng = np.random.default_rng(123)
+    ntok = inp.total_tokens
+    toks = np.concatenate([rng.integers(0, ntok, 120), [0, ntok - 1]])
+    # also the last token of every sequence (deepest Fenwick levels)
+    toks = np.concatenate([toks, [s + n - 1 for s, n in inp.seq_slices() if n > 0]])
+    samples = [(int(t), int(rng.integers(0, inp.H))) for t in toks]
+    ref = O.llattn_sampled(inp, samples)
+    got = run(inp, path="auto").reshape(-1, inp.H, inp.dv)
+    sel = np.stack([got[t, h] for t, h in samples])
+    assert np.isfinite(got).all()
+    err = O.rel_max_err(sel, ref)
+    assert err <= TOL[inp.dtype], f"{name}: sampled rel max err {err:.3e}"
