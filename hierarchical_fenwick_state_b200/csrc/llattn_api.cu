@@ -53,7 +53,7 @@ llattn_status resolve(int in_dtype, int* path, int* chunk, int T, int dk, int dv
   if (*path < LLATTN_PATH_AUTO || *path > LLATTN_PATH_TCGEN05) return LLATTN_ERR_ARG;
   if (*path == LLATTN_PATH_AUTO) {
     const int c = *chunk ? *chunk : default_chunk(LLATTN_PATH_TCGEN05, T);
-    *path = (in_dtype == LLATTN_BF16 && llattn::tc_supports(in_dtype, dk, dv, c))
+    *path = (in_dtype == LLATTN_BF16 && llattn::tc_supports(in_dtype, dk, dv, c, T))
                 ? LLATTN_PATH_TCGEN05 : LLATTN_PATH_SIMT;
   }
   if (*chunk == 0) *chunk = default_chunk(*path, T);
@@ -62,7 +62,7 @@ llattn_status resolve(int in_dtype, int* path, int* chunk, int T, int dk, int dv
     if (*chunk < 8 || *chunk > 64) return LLATTN_ERR_ARG;
   } else {
     if (in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
-    if (!llattn::tc_supports(in_dtype, dk, dv, *chunk)) return LLATTN_ERR_UNSUPPORTED;
+    if (!llattn::tc_supports(in_dtype, dk, dv, *chunk, T)) return LLATTN_ERR_UNSUPPORTED;
   }
   return LLATTN_OK;
 }
