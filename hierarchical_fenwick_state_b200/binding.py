@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libllattn.so")
 
 F32, BF16 = 0, 1
-PATHS = {"auto": 0, "simt": 1, "tcgen05": 2}
+PATHS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_serial": 3}
 
 # Every symbol include/llattn.h declares.
 EXPORTS = (

@@ -43,14 +43,14 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 int default_chunk(int path, int T) {
-  if (path == LLATTN_PATH_TCGEN05) return 128;
+  if (path == LLATTN_PATH_TCGEN05 || path == LLATTN_PATH_TCGEN05_SERIAL) return 128;
   return T <= 256 ? 16 : 64;
 }
 
 // Resolve AUTO, the chunk length, and check that the chosen path takes the shape.
 llattn_status resolve(int in_dtype, int* path, int* chunk, int T, int dk, int dv) {
   if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
-  if (*path < LLATTN_PATH_AUTO || *path > LLATTN_PATH_TCGEN05) return LLATTN_ERR_ARG;
+  if (*path < LLATTN_PATH_AUTO || *path > LLATTN_PATH_TCGEN05_SERIAL) return LLATTN_ERR_ARG;
   if (*path == LLATTN_PATH_AUTO) {
     const int c = *chunk ? *chunk : default_chunk(LLATTN_PATH_TCGEN05, T);
     *path = (in_dtype == LLATTN_BF16 && llattn::tc_supports(in_dtype, dk, dv, c, T))
@@ -152,8 +152,9 @@ llattn_status forward(int in_dtype, int path, int chunk, const void* q, const vo
   llattn::Problem p{in_dtype, q, k, v, log_a, lam, out, B, H, T, dk, dv, L, cu_seqlens,
                     ds->status};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = path == LLATTN_PATH_SIMT ? llattn::simt_forward(p, chunk, ws, st)
-                                           : llattn::tc_forward(p, chunk, ws, st);
+  cudaError_t e = path == LLATTN_PATH_SIMT
+                      ? llattn::simt_forward(p, chunk, ws, st)
+                      : llattn::tc_forward(p, chunk, ws, st, path == LLATTN_PATH_TCGEN05_SERIAL);
   if (e != cudaSuccess) return cuda_fail(e);
   return LLATTN_OK;
 }

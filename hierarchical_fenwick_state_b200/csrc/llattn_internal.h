@@ -34,7 +34,7 @@ size_t tc_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk);
 
 // Kernel launchers; return a cudaError_t from the launches.
 cudaError_t simt_forward(const Problem& p, int chunk, void* ws, cudaStream_t st);
-cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st);
+cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, bool serial);
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T);
 
 // Number of chunk-level Fenwick blocks kept per (sequence, head) for Nc chunks,

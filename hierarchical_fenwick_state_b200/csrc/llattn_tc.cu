@@ -96,7 +96,7 @@ __device__ __forceinline__ float bf16_at(const uint8_t* p) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+tc_fwd_serial(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
            const __grid_constant__ CUtensorMap tmv, const __nv_bfloat16* __restrict__ q,
            const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
            const float* __restrict__ log_a, const float* __restrict__ lam,
@@ -117,7 +117,7 @@ tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUte
   const int nch = (sp.len + kC - 1) / kC;
   const int LS = L | 1;              // odd row stride of the lam table: conflict-free
 
-  uint8_t* stage[2] = {sm, sm + kStage};
+  auto stage = [sm](int i) { return sm + i * kStage; };
   uint8_t* klo = sm + kOffKlo;
   uint8_t* slots = sm + kOffSlots;
   float* lamrow = reinterpret_cast<float*>(sm + kOffLam);
@@ -148,9 +148,9 @@ tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUte
   auto issue_load = [&](int c, int s) {
     const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
     mbar_arrive_expect_tx(&bars[s], 3 * kTile);
-    tma_load_3d(stage[s], &tmq, &bars[s], 0, h, tok0);
-    tma_load_3d(stage[s] + kTile, &tmk, &bars[s], 0, h, tok0);
-    tma_load_3d(stage[s] + 2 * kTile, &tmv, &bars[s], 0, h, tok0);
+    tma_load_3d(stage(s), &tmq, &bars[s], 0, h, tok0);
+    tma_load_3d(stage(s) + kTile, &tmk, &bars[s], 0, h, tok0);
+    tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[s], 0, h, tok0);
   };
   auto fail = [&]() {
     atomicOr(status, LLATTN_DEV_WAIT_TIMEOUT);
@@ -209,7 +209,7 @@ tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUte
           const int col = hf * 32 + j * 8;
           uint4 val = make_uint4(0u, 0u, 0u, 0u);
           if (row < n) val = *reinterpret_cast<const uint4*>(src + ((tok0 + row) * H + h) * kD + col);
-          *reinterpret_cast<uint4*>(stage[s] + tsr * kTile + sw128_off(row, col)) = val;
+          *reinterpret_cast<uint4*>(stage(s) + tsr * kTile + sw128_off(row, col)) = val;
         }
       }
       fence_proxy_async_smem();
@@ -240,7 +240,7 @@ tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUte
     __syncthreads();
 
     // ---- MMA issue: S = Q K^T, level readouts R_b = Q (S_b hi + S_b lo) ----
-    const uint32_t qa = smem_u32(stage[s]);
+    const uint32_t qa = smem_u32(stage(s));
     const uint32_t ka = qa + kTile;
     const uint32_t va = qa + 2 * kTile;
     int nlive = 0;
@@ -332,7 +332,7 @@ tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUte
     // ---- chunk state operand (a2): K rows scaled by exp(G - g_s), split hi (in place) / lo ----
     {
       const float ks = row < n ? __expf(gend - g_row) : 0.f;
-      uint8_t* kt = stage[s] + kTile;
+      uint8_t* kt = stage(s) + kTile;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t off = sw128_off(row, hf * 32 + j * 8);
@@ -491,6 +491,584 @@ tc_fwd_d64(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUte
   }
 }
 
+// ==========================================================================================
+// Pipelined variant: warp-specialised roles linked by mbarriers.
+//   warp 0        TMA producer (Q, K, V tiles of chunk c into stage c % 2)
+//   warp 1        MMA issuer   (S, H^T, level readouts, P V)
+//   warps 2..9    group A      (decay scan, K scaling for the chunk state, causal mask -> P)
+//   warps 10..17  group B      (Fenwick merge of the chunk state, epilogue and store)
+// S/P is double-buffered in TMEM, so group A masks chunk c+1 while group B finishes c.
+// P overwrites S in place, 16 keys at a time: the 16 fp32 columns of keys 16g..16g+15
+// become 8 columns of bf16 pairs (hi) followed by 8 (lo), so no thread ever writes
+// columns that it or another thread has still to read.
+// ==========================================================================================
+constexpr int kPW = 18;                       // warps
+constexpr int kPThreads = kPW * 32;
+constexpr int kPA0 = 2;                       // first warp of group A
+constexpr int kPNA = 8 * 32;                  // group A threads
+constexpr int kPB0 = 10;                      // first warp of group B
+constexpr int kPNB = 8 * 32;                  // group B threads
+
+constexpr uint32_t kPOffKlo = 2 * kStage;
+constexpr uint32_t kPOffSlots = kPOffKlo + kTile;
+constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
+constexpr uint32_t kPOffLam = kPOffSlots + kLevels * kSlot;
+constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[2][128]
+constexpr uint32_t kPOffCj = kPOffG + 2 * kC * 4;
+constexpr uint32_t kPOffScan = kPOffCj + kC * 4;
+constexpr uint32_t kPOffBar = kPOffScan + 64;
+constexpr int kPNumBars = 26;
+constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
+constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
+
+constexpr uint32_t kPColSP = 0;    // S/P buffer s at 128 * s
+constexpr uint32_t kPColO = 256;   // P V accumulator
+constexpr uint32_t kPColH = 320;   // H^T = V^T K_s, rows duplicated in lanes 64..127
+constexpr uint32_t kPColR = 384;   // two readout accumulators of 64 columns
+
+constexpr uint32_t kIdescHT = idesc_bf16(128, 64, 1, 1);  // V^T (M contiguous) x K_s (N contiguous)
+
+enum : int {
+  B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_SPEMPTY = 8, B_KS = 10, B_HFULL = 11,
+  B_HEMPTY = 12, B_LV = 13, B_OFULL = 14, B_OEMPTY = 15, B_RFULL = 16, B_REMPTY = 18,
+  B_GREADY = 20, B_GEMPTY = 22, B_DRAIN = 24, B_LV1 = 25
+};
+
+// Wait on an mbarrier phase; returns false at once if the CTA has aborted, and aborts
+// the CTA (flag + device status bit) if the wait exceeds its time limit.
+__device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, uint32_t* abort_flag,
+                                      unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  volatile uint32_t* ab = abort_flag;
+  if (*ab) return false;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*ab) return false;
+    if (globaltimer_ns() - t0 > 2000000000ull) {
+      atomicOr(status, LLATTN_DEV_WAIT_TIMEOUT);
+      *ab = 1u;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// MN-major descriptor whose second 64-row group along M repeats the first (LBO = 0):
+// an M = 128 MMA over a 64-wide operand yields the 64-row result twice.
+__device__ __forceinline__ uint64_t mndesc_dup(uint32_t saddr) { return sdesc_sw128(saddr, 0, 1024); }
+
+__global__ void __maxnreg__(96)
+tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+            const __grid_constant__ CUtensorMap tmv, const __nv_bfloat16* __restrict__ q,
+            const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+            const float* __restrict__ log_a, const float* __restrict__ lam,
+            float* __restrict__ out, int H, int T, int L, const int* __restrict__ cu,
+            unsigned int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int sub = warp & 3;
+  const int row = sub * 32 + lane;
+  const uint32_t lane_off = uint32_t(sub * 32) << 16;
+  const int h = blockIdx.x, sq = blockIdx.y;
+
+  const SeqSpan sp = seq_span(sq, T, cu, status);
+  if (sp.len <= 0) return;
+  const int nch = (sp.len + kC - 1) / kC;
+
+  auto stage = [sm](int i) { return sm + i * kStage; };
+  uint8_t* klo = sm + kPOffKlo;
+  uint8_t* slots = sm + kPOffSlots;
+  float* lamA = reinterpret_cast<float*>(sm + kPOffLam);
+  float* gs = reinterpret_cast<float*>(sm + kPOffG);
+  float* cj = reinterpret_cast<float*>(sm + kPOffCj);
+  float* scan = reinterpret_cast<float*>(sm + kPOffScan);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kPOffBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kPOffMisc);  // [0] TMEM base, [1] abort
+  uint32_t* abort_flag = &misc[1];
+
+  if (warp == 0) {
+    tmem_alloc(&misc[0], 512);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int i = 0; i < kPNumBars; ++i) {
+      uint32_t cnt = 1;  // TMA / tcgen05.commit arrivals
+      if (i == B_PFULL || i == B_PFULL + 1 || i == B_KS || i == B_GREADY || i == B_GREADY + 1)
+        cnt = kPNA;
+      if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY || i == B_REMPTY ||
+          i == B_REMPTY + 1 || i == B_GEMPTY || i == B_GEMPTY + 1)
+        cnt = kPNB;
+      mbar_init(&bars[i], cnt);
+    }
+    fence_mbar_init();
+    misc[1] = 0;
+    prefetch_tensormap(&tmq);
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  auto W = [&](int b, uint32_t parity) { return pwait(&bars[b], parity, abort_flag, status); };
+  auto is_full = [&](int c) { return (c + 1) * kC <= sp.len; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last0 = -1, last1 = -1;
+      for (int c = 0; c < nch && is_full(c); ++c) {
+        const int s = c & 1, kk = c >> 1;
+        if (!W(B_EMPTY + s, (kk & 1) ^ 1)) break;
+        const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
+        mbar_arrive_expect_tx(&bars[B_FULL + s], 3 * kTile);
+        tma_load_3d(stage(s), &tmq, &bars[B_FULL + s], 0, h, tok0);
+        tma_load_3d(stage(s) + kTile, &tmk, &bars[B_FULL + s], 0, h, tok0);
+        tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[B_FULL + s], 0, h, tok0);
+        if (s == 0) last0 = c; else last1 = c;
+      }
+      if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) {
+        // an aborted CTA still lets its own copies land before it exits
+        if (last0 >= 0) mbar_wait(&bars[B_FULL + 0], (last0 >> 1) & 1, 200000000ull);
+        if (last1 >= 0) mbar_wait(&bars[B_FULL + 1], (last1 >> 1) & 1, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t u = 0;  // readout accumulator uses so far (ring of two)
+      auto issue_S = [&](int c) -> bool {
+        const int s = c & 1, kk = c >> 1;
+        if (!W(B_FULL + s, kk & 1)) return false;
+        if (!W(B_SPEMPTY + s, (kk & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile;
+#pragma unroll
+        for (int x = 0; x < kD / 16; ++x)
+          mma_ss(tmem + kPColSP + 128 * s, kdesc(qa + x * 32), kdesc(ka + x * 32), kIdescS, x > 0);
+        mma_commit(&bars[B_SFULL + s]);
+        return true;
+      };
+      bool ok = issue_S(0);
+      // Per chunk c the issuer owes: H(c) (if a merge follows), the readouts R_b(c) for the
+      // set bits of c, P V(c) and S(c + 1).  It issues whichever is ready, testing barriers
+      // without blocking; all waits of one chunk are done before the next chunk starts,
+      // which keeps every barrier at most one phase ahead of its waiter.
+      for (int c = 0; ok && c < nch; ++c) {
+        const int s = c & 1, kk = c >> 1;
+        const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile, va = qa + 2 * kTile;
+        bool need_h = c + 1 < nch, need_pv = true, need_s = c + 1 < nch;
+        int next_b = 0;  // next level to read out
+        while (next_b < kLevels && !((c >> next_b) & 1)) ++next_b;
+        uint64_t t_idle = 0;
+        while (need_h || next_b < kLevels || need_pv || need_s) {
+          bool progress = false;
+          if (next_b < kLevels) {
+            const int rs = u & 1;
+            const bool lv_ok = c == 0 || mbar_test(&bars[((c - 1) & 1) ? B_LV1 : B_LV], ((c - 1) >> 1) & 1);
+            if (lv_ok && mbar_test(&bars[B_REMPTY + rs], ((u >> 1) & 1) ^ 1)) {
+              tc_fence_after();
+              const uint32_t d = tmem + kPColR + 64 * rs;
+              const uint32_t sb = smem_u32(slots + next_b * kSlot);
+#pragma unroll
+              for (int x = 0; x < kD / 16; ++x)
+                mma_ss(d, kdesc(qa + x * 32), kdesc(sb + x * 32), kIdescR, x > 0);
+#pragma unroll
+              for (int x = 0; x < kD / 16; ++x)
+                mma_ss(d, kdesc(qa + x * 32), kdesc(sb + 8192 + x * 32), kIdescR, 1);
+              mma_commit(&bars[B_RFULL + rs]);
+              ++u;
+              ++next_b;
+              while (next_b < kLevels && !((c >> next_b) & 1)) ++next_b;
+              progress = true;
+            }
+          }
+          if (need_h && mbar_test(&bars[B_KS], c & 1) && mbar_test(&bars[B_HEMPTY], (c & 1) ^ 1)) {
+            tc_fence_after();
+            const uint32_t kl = smem_u32(klo);
+#pragma unroll
+            for (int x = 0; x < kC / 16; ++x)
+              mma_ss(tmem + kPColH, mndesc_dup(va + x * 2048), mndesc(ka + x * 2048), kIdescHT, x > 0);
+#pragma unroll
+            for (int x = 0; x < kC / 16; ++x)
+              mma_ss(tmem + kPColH, mndesc_dup(va + x * 2048), mndesc(kl + x * 2048), kIdescHT, 1);
+            mma_commit(&bars[B_HFULL]);
+            need_h = false;
+            progress = true;
+          }
+          if (need_pv && mbar_test(&bars[B_PFULL + s], kk & 1) &&
+              mbar_test(&bars[B_OEMPTY], (c & 1) ^ 1)) {
+            tc_fence_after();
+            const uint32_t spc = tmem + kPColSP + 128 * s;
+            // K-step x covers keys 16x..16x+15: hi in columns 16x..16x+7, lo in 16x+8..16x+15
+#pragma unroll
+            for (int x = 0; x < kC / 16; ++x)
+              mma_ts(tmem + kPColO, spc + 16 * x, mndesc(va + x * 2048), kIdescPV, x > 0);
+#pragma unroll
+            for (int x = 0; x < kC / 16; ++x)
+              mma_ts(tmem + kPColO, spc + 16 * x + 8, mndesc(va + x * 2048), kIdescPV, 1);
+            mma_commit(&bars[B_OFULL]);
+            mma_commit(&bars[B_SPEMPTY + s]);
+            need_pv = false;
+            progress = true;
+          }
+          if (need_s) {
+            const int s1 = (c + 1) & 1, k1 = (c + 1) >> 1;
+            if (mbar_test(&bars[B_FULL + s1], k1 & 1) &&
+                mbar_test(&bars[B_SPEMPTY + s1], (k1 & 1) ^ 1)) {
+              tc_fence_after();
+              const uint32_t q1 = smem_u32(stage(s1)), k1a = q1 + kTile;
+#pragma unroll
+              for (int x = 0; x < kD / 16; ++x)
+                mma_ss(tmem + kPColSP + 128 * s1, kdesc(q1 + x * 32), kdesc(k1a + x * 32), kIdescS, x > 0);
+              mma_commit(&bars[B_SFULL + s1]);
+              need_s = false;
+              progress = true;
+            }
+          }
+          if (progress) {
+            t_idle = 0;
+          } else {
+            if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) { ok = false; break; }
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) {
+              t_idle = now;
+            } else if (now - t_idle > 2000000000ull) {
+              atomicOr(status, LLATTN_DEV_WAIT_TIMEOUT);
+              *reinterpret_cast<volatile uint32_t*>(abort_flag) = 1u;
+              ok = false;
+              break;
+            }
+            __nanosleep(32);
+          }
+        }
+        // stage s is free once every MMA that reads it (S, H, readouts, P V) has completed;
+        // only now are all of them issued
+        if (ok) mma_commit(&bars[B_EMPTY + s]);
+      }
+      mma_commit(&bars[B_DRAIN]);
+      mbar_wait(&bars[B_DRAIN], 0, 200000000ull);
+    }
+  } else if (warp < kPB0) {
+    // ------------------------------------------------------------ group A
+    const int wa = warp - kPA0;     // 0..7
+    const int part = wa >> 2;       // column blocks part, part + 2; K columns 32*part..
+    float pf[4];
+    float pf_la = 0.f;
+    auto prefetch = [&](int c) {
+      const int t = c * kC + row;
+      const bool okt = t < sp.len;
+      const long long tok = sp.start + t;
+      const float* lr = lam + (tok * H + h) * L;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int l = part + 2 * i;
+        pf[i] = (okt && l < L) ? __ldg(lr + l) : 0.f;
+      }
+      if (part == 0) pf_la = okt ? __ldg(log_a + tok * H + h) : 0.f;
+    };
+    prefetch(0);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1, kk = c >> 1;
+      const int n = min(kC, sp.len - c * kC);
+      float pfc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pfc[i] = pf[i];
+      const float la = pf_la;
+      if (c + 1 < nch) prefetch(c + 1);
+      W(B_GEMPTY + s, (kk & 1) ^ 1);   // group B is done with g[s] of chunk c - 2
+      float x = la;
+      if (part == 0) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) scan[sub] = x;
+      }
+      named_sync(1, kPNA);  // also: every mask read of the previous chunk is done
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lamA[row * kPLamStride + part + 2 * i] = pfc[i];
+      if (part == 0) {
+        float off = 0.f;
+        for (int w = 0; w < sub; ++w) off += scan[w];
+        gs[s * kC + row] = x + off;
+      }
+      named_sync(1, kPNA);
+      const float g_row = gs[s * kC + row];
+      const float g0 = gs[s * kC];
+      const float gend = gs[s * kC + n - 1];
+      const bool factored = (g0 - gend) <= 80.f;
+      if (part == 0) cj[row] = factored ? __expf(g0 - g_row) : 0.f;
+      mbar_arrive(&bars[B_GREADY + s]);
+      if (!is_full(c)) {
+        // ragged last chunk: plain loads into the stage, rows past the end zero-filled
+        W(B_EMPTY + s, (kk & 1) ^ 1);
+        const long long tok0 = sp.start + (long long)c * kC;
+#pragma unroll
+        for (int tsr = 0; tsr < 3; ++tsr) {
+          const __nv_bfloat16* src = tsr == 0 ? q : (tsr == 1 ? k : v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int col = part * 32 + j * 8;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (row < n)
+              val = *reinterpret_cast<const uint4*>(src + ((tok0 + row) * H + h) * kD + col);
+            *reinterpret_cast<uint4*>(stage(s) + tsr * kTile + sw128_off(row, col)) = val;
+          }
+        }
+        fence_proxy_async_smem();
+        named_sync(1, kPNA);
+        if (wa == 0 && lane == 0) mbar_arrive(&bars[B_FULL + s]);
+      }
+      W(B_FULL + s, kk & 1);
+      W(B_SFULL + s, kk & 1);
+      tc_fence_after();
+      named_sync(1, kPNA);  // cj and the lam table are visible to the whole group
+      // ---- chunk-state operand: K rows scaled by exp(G - g_s), hi in place, lo to klo ----
+      if (c + 1 < nch) {
+        if (c > 0) W(B_HFULL, (c - 1) & 1);   // H of the previous chunk has read klo
+        const float ks = row < n ? __expf(gend - g_row) : 0.f;
+        uint8_t* kt = stage(s) + kTile;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t off = sw128_off(row, part * 32 + j * 8);
+          const uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
+          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
+            split_pack(__low2float(pr) * ks, __high2float(pr) * ks, hi[e], lo[e]);
+          }
+          *reinterpret_cast<uint4*>(kt + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(klo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[B_KS]);
+      }
+      // ---- causal Fenwick mask on S -> P (hi/lo), one 32-key block at a time ----
+      const uint32_t spc = tmem + lane_off + kPColSP + 128 * s;
+      const int rb = sub;
+      const float ri = factored ? __expf(g_row - g0) : 0.f;
+      const float* lr = lamA + row * kPLamStride;
+#pragma unroll 1
+      for (int kb = part; kb < 4; kb += 2) {
+        if (kb > rb) {
+          uint32_t z[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) z[e] = 0u;
+          tmem_st16(spc + 32 * kb, z);
+          tmem_st16(spc + 32 * kb + 16, z);
+          continue;
+        }
+        const float rsc = factored ? ri : 1.f;
+        // off-diagonal blocks have one Fenwick level; the diagonal block one per element
+        const float wblk = kb < rb ? lr[6 + (31 - __clz(rb ^ kb))] * rsc : 0.f;
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const int g16 = 2 * kb + hh;  // keys 16*g16 .. 16*g16+15
+          float sv[16];
+          tmem_ld16(spc + 16 * g16, sv);
+          tmem_wait_ld();
+          // weight of key j: (lam x exp(g_i - g_0)) x exp(g_0 - g_j) when that stays finite,
+          // else lam x exp(g_i - g_j) element by element
+          float cw[16];
+          if (factored) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(cj + 16 * g16 + e);
+              cw[e] = c4.x; cw[e + 1] = c4.y; cw[e + 2] = c4.z; cw[e + 3] = c4.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) cw[e] = __expf(g_row - gs[s * kC + 16 * g16 + e]);
+          }
+          uint32_t hi[8], lo[8];
+          if (kb < rb) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 2)
+              split_pack(sv[e] * wblk * cw[e], sv[e + 1] * wblk * cw[e + 1], hi[e >> 1], lo[e >> 1]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              float p[2];
+#pragma unroll
+              for (int t2 = 0; t2 < 2; ++t2) {
+                const int jj = 16 * hh + e + t2;  // key index inside the 32-key block
+                const int lev = (jj == lane) ? 0 : (32 - __clz(jj ^ lane));
+                const float val = sv[e + t2] * (lr[lev] * rsc) * cw[e + t2];
+                p[t2] = jj <= lane ? val : 0.f;
+              }
+              split_pack(p[0], p[1], hi[e >> 1], lo[e >> 1]);
+            }
+          }
+          tmem_st8(spc + 16 * g16, hi);
+          tmem_st8(spc + 16 * g16 + 8, lo);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[B_PFULL + s]);
+    }
+  } else {
+    // ------------------------------------------------------------ group B
+    const int half = (warp - kPB0) >> 2;   // which 32 of the 64 output columns
+    const int j_dv = row & 63;             // merge: row of H^T (a d_v index) ...
+    const int dk0 = 32 * (row >> 6) + 16 * half;  // ... and the 16 d_k columns it merges
+    float pl[kLevels];
+    auto prefetch = [&](int c) {
+      const int t = c * kC + row;
+      const bool okt = t < sp.len;
+      const long long tok = sp.start + t;
+      const float* lr = lam + (tok * H + h) * L;
+#pragma unroll
+      for (int b = 0; b < kLevels; ++b) {
+        const int l = 1 + kLogC + b;
+        pl[b] = (okt && l < L && ((c >> b) & 1)) ? __ldg(lr + l) : 0.f;
+      }
+    };
+    prefetch(0);
+    float gtot[kLevels];
+#pragma unroll
+    for (int b = 0; b < kLevels; ++b) gtot[b] = 0.f;
+    uint32_t u = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1, kk = c >> 1;
+      const int n = min(kC, sp.len - c * kC);
+      W(B_GREADY + s, kk & 1);
+      const float g_row = gs[s * kC + row];
+      const float gend = gs[s * kC + n - 1];
+      float lamv[kLevels];
+#pragma unroll
+      for (int b = 0; b < kLevels; ++b) lamv[b] = pl[b];
+      if (c + 1 < nch) prefetch(c + 1);
+      // ---- epilogue: o = sum_b lam[., 1+log2 C+b] exp(g + gap_b) R_b + P V ----
+      // The readouts are drained first: the MMA warp issues them before P V and may be
+      // waiting for a free readout accumulator.
+      float o[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+      float gap = 0.f;
+#pragma unroll
+      for (int b = 0; b < kLevels; ++b) {
+        if (!((c >> b) & 1)) continue;
+        const int rs = u & 1;
+        W(B_RFULL + rs, (u >> 1) & 1);
+        tc_fence_after();
+        const float w = lamv[b] * __expf(g_row + gap);
+        float r0[32];
+        tmem_ld32(tmem + lane_off + kPColR + 64 * rs + 32 * half, r0);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars[B_REMPTY + rs]);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = fmaf(w, r0[e], o[e]);
+        gap += gtot[b];
+        ++u;
+      }
+      // ---- Fenwick merge: level m = H + sum_{b<m} exp(decay after block b) S_b ----
+      if (c + 1 < nch) {
+        const int m = __ffs(~c) - 1;
+        // the lower levels do not depend on this chunk: sum them before H arrives
+        float hv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) hv[e] = 0.f;
+        float acc = gend;
+#pragma unroll
+        for (int b = 0; b < kLevels; ++b) {
+          if (b < m) {
+            const float f = __expf(acc);
+            const uint8_t* sl = slots + b * kSlot;
+#pragma unroll
+            for (int qd = 0; qd < 2; ++qd) {
+              const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
+              const uint4 a4 = *reinterpret_cast<const uint4*>(sl + off);
+              const uint4 b4 = *reinterpret_cast<const uint4*>(sl + 8192 + off);
+              const uint32_t av[4] = {a4.x, a4.y, a4.z, a4.w};
+              const uint32_t bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 ah = *reinterpret_cast<const __nv_bfloat162*>(&av[e]);
+                const __nv_bfloat162 bl = *reinterpret_cast<const __nv_bfloat162*>(&bv[e]);
+                hv[8 * qd + 2 * e] = fmaf(f, __low2float(ah) + __low2float(bl), hv[8 * qd + 2 * e]);
+                hv[8 * qd + 2 * e + 1] =
+                    fmaf(f, __high2float(ah) + __high2float(bl), hv[8 * qd + 2 * e + 1]);
+              }
+            }
+            acc += gtot[b];
+          }
+        }
+        W(B_HFULL, c & 1);
+        tc_fence_after();
+        {
+          float t16[16];
+          tmem_ld16(tmem + lane_off + kPColH + 32 * (row >> 6) + 16 * half, t16);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) hv[e] += t16[e];
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[B_HEMPTY]);
+        uint8_t* dsl = slots + m * kSlot;
+#pragma unroll
+        for (int qd = 0; qd < 2; ++qd) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            split_pack(hv[8 * qd + 2 * e], hv[8 * qd + 2 * e + 1], hi[e], lo[e]);
+          const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
+          *reinterpret_cast<uint4*>(dsl + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(dsl + 8192 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_proxy_async_smem();
+#pragma unroll
+        for (int b = 0; b < kLevels; ++b)
+          if (b == m) gtot[b] = acc;
+        mbar_arrive(&bars[(c & 1) ? B_LV1 : B_LV]);
+      }
+      W(B_OFULL, c & 1);
+      tc_fence_after();
+      {
+        float r0[32];
+        tmem_ld32(tmem + lane_off + kPColO + 32 * half, r0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] += r0[e];
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_OEMPTY]);
+      if (row < n) {
+        float* dst = out + ((sp.start + (long long)c * kC + row) * H + h) * kD + 32 * half;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+      }
+      mbar_arrive(&bars[B_GEMPTY + s]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -534,7 +1112,7 @@ bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T) {
 
 size_t tc_workspace_bytes(int, int, int, int, int, int) { return 0; }
 
-cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st) {
+cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool serial) {
   if (!tc_supports(p.in_dtype, p.dk, p.dv, chunk, p.T)) return cudaErrorNotSupported;
   // TMA only ever fetches whole chunks inside a sequence, so the token extent can be
   // the dense size, or for packed batches any bound >= the real total (nseq * T).
@@ -547,17 +1125,25 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st) {
   if ((e = make_map(&mv, p.v, p.H, tokens)) != cudaSuccess) return e;
   static bool attr_set = false;
   if (!attr_set) {
-    if ((e = cudaFuncSetAttribute(tc_fwd_d64, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(tc_fwd_serial, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kSmemBytes)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(tc_fwd_pipe, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kPSmemBytes)) != cudaSuccess)
       return e;
     attr_set = true;
   }
   const dim3 grid(p.H, p.nseq);
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(p.k);
+  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(p.v);
   main_kernel_begin(st);
-  tc_fwd_d64<<<grid, kThreads, kSmemBytes, st>>>(
-      mq, mk, mv, static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
-      static_cast<const __nv_bfloat16*>(p.v), p.log_a, p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens,
-      p.status);
+  if (serial)
+    tc_fwd_serial<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, q, k, v, p.log_a, p.lam, p.out,
+                                                      p.H, p.T, p.L, p.cu_seqlens, p.status);
+  else
+    tc_fwd_pipe<<<grid, kPThreads, kPSmemBytes, st>>>(mq, mk, mv, q, k, v, p.log_a, p.lam, p.out,
+                                                      p.H, p.T, p.L, p.cu_seqlens, p.status);
   main_kernel_end(st);
   count_launch();
   return cudaGetLastError();

@@ -76,10 +76,17 @@ typedef enum {
 enum { LLATTN_F32 = 0, LLATTN_BF16 = 1 };
 
 /* Kernel paths for llattn_fwd_ex.
- *   AUTO     tcgen05 path where one exists for the shape, else SIMT.
- *   SIMT     CUDA-core kernels (any dk, dv in {32,64,128}; fp32 or bf16 inputs).
- *   TCGEN05  tensor-core kernels (bf16 inputs only). */
-enum { LLATTN_PATH_AUTO = 0, LLATTN_PATH_SIMT = 1, LLATTN_PATH_TCGEN05 = 2 };
+ *   AUTO            tcgen05 path where one exists for the shape, else SIMT.
+ *   SIMT            CUDA-core kernels (any dk, dv in {32,64,128}; fp32 or bf16 inputs).
+ *   TCGEN05         tensor-core kernel, warp-specialised pipeline (bf16 inputs only).
+ *   TCGEN05_SERIAL  the same arithmetic with one warp group walking each chunk's steps in
+ *                   order (a slower cross-check of the pipelined kernel). */
+enum {
+  LLATTN_PATH_AUTO = 0,
+  LLATTN_PATH_SIMT = 1,
+  LLATTN_PATH_TCGEN05 = 2,
+  LLATTN_PATH_TCGEN05_SERIAL = 3
+};
 
 /* Device status bits (llattn_device_status). */
 enum {

@@ -26,7 +26,7 @@ def _paths_for(inp):
         try:
             binding.workspace_bytes(1, "tcgen05", 0, inp.B, inp.H, inp.T, inp.dk, inp.dv,
                                     inp.cu_seqlens is not None)
-            paths.append("tcgen05")
+            paths += ["tcgen05", "tcgen05_serial"]
         except binding.LLAttnError:
             pass
     return paths
