@@ -103,8 +103,9 @@ tc_fwd_serial(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
            float* __restrict__ out, int H, int T, int L, const int* __restrict__ cu,
            unsigned int* status) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+  // 1024-byte aligned base, by pointer arithmetic on the shared array so that the compiler
+  // keeps shared-memory (not generic) loads and stores for everything derived from it
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = warp & 3;          // TMEM sub-partition: lanes 32*sub .. 32*sub+31
   const int hf = warp >> 2;          // which 32/64-column half of a row this thread handles
@@ -494,44 +495,49 @@ tc_fwd_serial(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
 // ==========================================================================================
 // Pipelined variant: warp-specialised roles linked by mbarriers.
 //   warp 0        TMA producer (Q, K, V tiles of chunk c into stage c % 2)
-//   warp 1        MMA issuer   (S, H^T, level readouts, P V)
+//   warp 1        MMA issuer for the intra-chunk part (S, P V)
+//   warp 18       MMA issuer for the inter-chunk part (H^T, level readouts)
 //   warps 2..9    group A      (decay scan, K scaling for the chunk state, causal mask -> P)
 //   warps 10..17  group B      (Fenwick merge of the chunk state, epilogue and store)
-// S/P is double-buffered in TMEM, so group A masks chunk c+1 while group B finishes c.
+// TMEM holds S/P, the P V accumulator, H^T and four level-readout accumulators, so a
+// chunk's readouts (up to four levels at once) are in flight together.
 // P overwrites S in place, 16 keys at a time: the 16 fp32 columns of keys 16g..16g+15
 // become 8 columns of bf16 pairs (hi) followed by 8 (lo), so no thread ever writes
 // columns that it or another thread has still to read.
 // ==========================================================================================
-constexpr int kPW = 18;                       // warps
+constexpr int kPW = 19;                       // warps
 constexpr int kPThreads = kPW * 32;
 constexpr int kPA0 = 2;                       // first warp of group A
 constexpr int kPNA = 8 * 32;                  // group A threads
 constexpr int kPB0 = 10;                      // first warp of group B
 constexpr int kPNB = 8 * 32;                  // group B threads
+constexpr int kPI2 = 18;                      // warp of the inter-chunk MMA issuer
 
 constexpr uint32_t kPOffKlo = 2 * kStage;
-constexpr uint32_t kPOffSlots = kPOffKlo + kTile;
+constexpr uint32_t kPOffSlots = kPOffKlo + kTile;   // level hi parts, then level lo parts
+constexpr uint32_t kPLoOff = kLevels * 8192;        // lo part of level b at + kPLoOff + b * 8 KB
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
 constexpr uint32_t kPOffLam = kPOffSlots + kLevels * kSlot;
 constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[2][128]
 constexpr uint32_t kPOffCj = kPOffG + 2 * kC * 4;
 constexpr uint32_t kPOffScan = kPOffCj + kC * 4;
 constexpr uint32_t kPOffBar = kPOffScan + 64;
-constexpr int kPNumBars = 26;
+constexpr int kPNumBars = 22;
 constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
 constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
 
-constexpr uint32_t kPColSP = 0;    // S/P buffer s at 128 * s
-constexpr uint32_t kPColO = 256;   // P V accumulator
-constexpr uint32_t kPColH = 320;   // H^T = V^T K_s, rows duplicated in lanes 64..127
-constexpr uint32_t kPColR = 384;   // two readout accumulators of 64 columns
+constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (hi/lo)
+constexpr uint32_t kPColO = 128;   // P V accumulator
+constexpr uint32_t kPColH = 192;   // H^T = V^T K_s, rows duplicated in lanes 64..127
+constexpr uint32_t kPColR = 256;   // readout accumulator: up to four adjacent levels
+constexpr int kPSpan = 4;          // levels one readout chain covers (N = 64 per level)
 
 constexpr uint32_t kIdescHT = idesc_bf16(128, 64, 1, 1);  // V^T (M contiguous) x K_s (N contiguous)
 
 enum : int {
-  B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_SPEMPTY = 8, B_KS = 10, B_HFULL = 11,
-  B_HEMPTY = 12, B_LV = 13, B_OFULL = 14, B_OEMPTY = 15, B_RFULL = 16, B_REMPTY = 18,
-  B_GREADY = 20, B_GEMPTY = 22, B_DRAIN = 24, B_LV1 = 25
+  B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 5, B_SPEMPTY = 6, B_KS = 7, B_HFULL = 8,
+  B_HEMPTY = 9, B_LV = 10, B_LV1 = 11, B_OFULL = 12, B_OEMPTY = 13, B_RFULL = 14,
+  B_REMPTY = 15, B_GREADY = 16, B_GEMPTY = 18, B_DRAIN = 20, B_DRAIN2 = 21
 };
 
 // Wait on an mbarrier phase; returns false at once if the CTA has aborted, and aborts
@@ -564,6 +570,21 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// The readouts of one chunk go out in chains: a chain starts at the lowest remaining set
+// bit b0 of c and covers the set bits below b0 + kPSpan; its N = 64 * (b1 - b0 + 1)
+// columns read the consecutive hi (then lo) level arrays in one MMA per K step.  A level
+// inside the range whose bit is clear is computed and ignored.
+__device__ __forceinline__ bool next_chain(int c, int from, int& b0, int& b1) {
+  int b = from;
+  while (b < kLevels && !((c >> b) & 1)) ++b;
+  if (b >= kLevels) return false;
+  b0 = b;
+  b1 = b;
+  for (int x = b + 1; x < kLevels && x < b + kPSpan; ++x)
+    if ((c >> x) & 1) b1 = x;
+  return true;
+}
+
 // MN-major descriptor whose second 64-row group along M repeats the first (LBO = 0):
 // an M = 128 MMA over a 64-wide operand yields the 64-row result twice.
 __device__ __forceinline__ uint64_t mndesc_dup(uint32_t saddr) { return sdesc_sw128(saddr, 0, 1024); }
@@ -576,8 +597,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             float* __restrict__ out, int H, int T, int L, const int* __restrict__ cu,
             unsigned int* status) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+  // 1024-byte aligned base, by pointer arithmetic on the shared array so that the compiler
+  // keeps shared-memory (not generic) loads and stores for everything derived from it
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = warp & 3;
   const int row = sub * 32 + lane;
@@ -606,10 +628,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   if (tid == 32) {
     for (int i = 0; i < kPNumBars; ++i) {
       uint32_t cnt = 1;  // TMA / tcgen05.commit arrivals
-      if (i == B_PFULL || i == B_PFULL + 1 || i == B_KS || i == B_GREADY || i == B_GREADY + 1)
-        cnt = kPNA;
-      if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY || i == B_REMPTY ||
-          i == B_REMPTY + 1 || i == B_GEMPTY || i == B_GEMPTY + 1)
+      if (i == B_EMPTY || i == B_EMPTY + 1) cnt = 2;  // one commit from each MMA issuer
+      if (i == B_PFULL || i == B_KS || i == B_GREADY || i == B_GREADY + 1) cnt = kPNA;
+      if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY ||
+          i == B_REMPTY || i == B_GEMPTY || i == B_GEMPTY + 1)
         cnt = kPNB;
       mbar_init(&bars[i], cnt);
     }
@@ -647,117 +669,41 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ intra-chunk MMA issuer
+    // S(c) = Q K^T and P V(c); S(c + 1) overwrites P(c), so it follows P V(c).
     if (lane == 0) {
-      uint32_t u = 0;  // readout accumulator uses so far (ring of two)
-      auto issue_S = [&](int c) -> bool {
-        const int s = c & 1, kk = c >> 1;
-        if (!W(B_FULL + s, kk & 1)) return false;
-        if (!W(B_SPEMPTY + s, (kk & 1) ^ 1)) return false;
+      bool ok = W(B_FULL, 0);
+      if (ok) {
         tc_fence_after();
-        const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile;
+        const uint64_t qd = kdesc(smem_u32(stage(0))), kd = kdesc(smem_u32(stage(0)) + kTile);
 #pragma unroll
-        for (int x = 0; x < kD / 16; ++x)
-          mma_ss(tmem + kPColSP + 128 * s, kdesc(qa + x * 32), kdesc(ka + x * 32), kIdescS, x > 0);
-        mma_commit(&bars[B_SFULL + s]);
-        return true;
-      };
-      bool ok = issue_S(0);
-      // Per chunk c the issuer owes: H(c) (if a merge follows), the readouts R_b(c) for the
-      // set bits of c, P V(c) and S(c + 1).  It issues whichever is ready, testing barriers
-      // without blocking; all waits of one chunk are done before the next chunk starts,
-      // which keeps every barrier at most one phase ahead of its waiter.
+        for (int x = 0; x < kD / 16; ++x) mma_ss(tmem + kPColSP, qd + 2 * x, kd + 2 * x, kIdescS, x > 0);
+        mma_commit(&bars[B_SFULL]);
+      }
       for (int c = 0; ok && c < nch; ++c) {
-        const int s = c & 1, kk = c >> 1;
-        const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile, va = qa + 2 * kTile;
-        bool need_h = c + 1 < nch, need_pv = true, need_s = c + 1 < nch;
-        int next_b = 0;  // next level to read out
-        while (next_b < kLevels && !((c >> next_b) & 1)) ++next_b;
-        uint64_t t_idle = 0;
-        while (need_h || next_b < kLevels || need_pv || need_s) {
-          bool progress = false;
-          if (next_b < kLevels) {
-            const int rs = u & 1;
-            const bool lv_ok = c == 0 || mbar_test(&bars[((c - 1) & 1) ? B_LV1 : B_LV], ((c - 1) >> 1) & 1);
-            if (lv_ok && mbar_test(&bars[B_REMPTY + rs], ((u >> 1) & 1) ^ 1)) {
-              tc_fence_after();
-              const uint32_t d = tmem + kPColR + 64 * rs;
-              const uint32_t sb = smem_u32(slots + next_b * kSlot);
+        const int s = c & 1;
+        if (!W(B_PFULL, c & 1) || !W(B_OEMPTY, (c & 1) ^ 1)) break;
+        tc_fence_after();
+        // K-step x covers keys 16x..16x+15: hi in columns 16x..16x+7, lo in 16x+8..16x+15
+        const uint64_t vd = mndesc(smem_u32(stage(s)) + 2 * kTile);
 #pragma unroll
-              for (int x = 0; x < kD / 16; ++x)
-                mma_ss(d, kdesc(qa + x * 32), kdesc(sb + x * 32), kIdescR, x > 0);
+        for (int x = 0; x < kC / 16; ++x)
+          mma_ts(tmem + kPColO, tmem + kPColSP + 16 * x, vd + 128 * x, kIdescPV, x > 0);
 #pragma unroll
-              for (int x = 0; x < kD / 16; ++x)
-                mma_ss(d, kdesc(qa + x * 32), kdesc(sb + 8192 + x * 32), kIdescR, 1);
-              mma_commit(&bars[B_RFULL + rs]);
-              ++u;
-              ++next_b;
-              while (next_b < kLevels && !((c >> next_b) & 1)) ++next_b;
-              progress = true;
-            }
-          }
-          if (need_h && mbar_test(&bars[B_KS], c & 1) && mbar_test(&bars[B_HEMPTY], (c & 1) ^ 1)) {
-            tc_fence_after();
-            const uint32_t kl = smem_u32(klo);
+        for (int x = 0; x < kC / 16; ++x)
+          mma_ts(tmem + kPColO, tmem + kPColSP + 16 * x + 8, vd + 128 * x, kIdescPV, 1);
+        mma_commit(&bars[B_OFULL]);
+        mma_commit(&bars[B_SPEMPTY]);
+        mma_commit(&bars[B_EMPTY + s]);   // this issuer's reads of stage s are done
+        if (c + 1 < nch) {
+          const int s1 = (c + 1) & 1;
+          if (!W(B_FULL + s1, ((c + 1) >> 1) & 1) || !W(B_SPEMPTY, c & 1)) break;
+          tc_fence_after();
+          const uint64_t qd = kdesc(smem_u32(stage(s1))), kd = kdesc(smem_u32(stage(s1)) + kTile);
 #pragma unroll
-            for (int x = 0; x < kC / 16; ++x)
-              mma_ss(tmem + kPColH, mndesc_dup(va + x * 2048), mndesc(ka + x * 2048), kIdescHT, x > 0);
-#pragma unroll
-            for (int x = 0; x < kC / 16; ++x)
-              mma_ss(tmem + kPColH, mndesc_dup(va + x * 2048), mndesc(kl + x * 2048), kIdescHT, 1);
-            mma_commit(&bars[B_HFULL]);
-            need_h = false;
-            progress = true;
-          }
-          if (need_pv && mbar_test(&bars[B_PFULL + s], kk & 1) &&
-              mbar_test(&bars[B_OEMPTY], (c & 1) ^ 1)) {
-            tc_fence_after();
-            const uint32_t spc = tmem + kPColSP + 128 * s;
-            // K-step x covers keys 16x..16x+15: hi in columns 16x..16x+7, lo in 16x+8..16x+15
-#pragma unroll
-            for (int x = 0; x < kC / 16; ++x)
-              mma_ts(tmem + kPColO, spc + 16 * x, mndesc(va + x * 2048), kIdescPV, x > 0);
-#pragma unroll
-            for (int x = 0; x < kC / 16; ++x)
-              mma_ts(tmem + kPColO, spc + 16 * x + 8, mndesc(va + x * 2048), kIdescPV, 1);
-            mma_commit(&bars[B_OFULL]);
-            mma_commit(&bars[B_SPEMPTY + s]);
-            need_pv = false;
-            progress = true;
-          }
-          if (need_s) {
-            const int s1 = (c + 1) & 1, k1 = (c + 1) >> 1;
-            if (mbar_test(&bars[B_FULL + s1], k1 & 1) &&
-                mbar_test(&bars[B_SPEMPTY + s1], (k1 & 1) ^ 1)) {
-              tc_fence_after();
-              const uint32_t q1 = smem_u32(stage(s1)), k1a = q1 + kTile;
-#pragma unroll
-              for (int x = 0; x < kD / 16; ++x)
-                mma_ss(tmem + kPColSP + 128 * s1, kdesc(q1 + x * 32), kdesc(k1a + x * 32), kIdescS, x > 0);
-              mma_commit(&bars[B_SFULL + s1]);
-              need_s = false;
-              progress = true;
-            }
-          }
-          if (progress) {
-            t_idle = 0;
-          } else {
-            if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) { ok = false; break; }
-            const uint64_t now = globaltimer_ns();
-            if (t_idle == 0) {
-              t_idle = now;
-            } else if (now - t_idle > 2000000000ull) {
-              atomicOr(status, LLATTN_DEV_WAIT_TIMEOUT);
-              *reinterpret_cast<volatile uint32_t*>(abort_flag) = 1u;
-              ok = false;
-              break;
-            }
-            __nanosleep(32);
-          }
+          for (int x = 0; x < kD / 16; ++x) mma_ss(tmem + kPColSP, qd + 2 * x, kd + 2 * x, kIdescS, x > 0);
+          mma_commit(&bars[B_SFULL]);
         }
-        // stage s is free once every MMA that reads it (S, H, readouts, P V) has completed;
-        // only now are all of them issued
-        if (ok) mma_commit(&bars[B_EMPTY + s]);
       }
       mma_commit(&bars[B_DRAIN]);
       mbar_wait(&bars[B_DRAIN], 0, 200000000ull);
@@ -835,33 +781,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         if (wa == 0 && lane == 0) mbar_arrive(&bars[B_FULL + s]);
       }
       W(B_FULL + s, kk & 1);
-      W(B_SFULL + s, kk & 1);
+      W(B_SFULL, c & 1);
       tc_fence_after();
       named_sync(1, kPNA);  // cj and the lam table are visible to the whole group
-      // ---- chunk-state operand: K rows scaled by exp(G - g_s), hi in place, lo to klo ----
-      if (c + 1 < nch) {
-        if (c > 0) W(B_HFULL, (c - 1) & 1);   // H of the previous chunk has read klo
-        const float ks = row < n ? __expf(gend - g_row) : 0.f;
-        uint8_t* kt = stage(s) + kTile;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t off = sw128_off(row, part * 32 + j * 8);
-          const uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
-          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
-            split_pack(__low2float(pr) * ks, __high2float(pr) * ks, hi[e], lo[e]);
-          }
-          *reinterpret_cast<uint4*>(kt + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(klo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&bars[B_KS]);
-      }
       // ---- causal Fenwick mask on S -> P (hi/lo), one 32-key block at a time ----
-      const uint32_t spc = tmem + lane_off + kPColSP + 128 * s;
+      const uint32_t spc = tmem + lane_off + kPColSP;
       const int rb = sub;
       const float ri = factored ? __expf(g_row - g0) : 0.f;
       const float* lr = lamA + row * kPLamStride;
@@ -922,9 +846,33 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_PFULL + s]);
+      mbar_arrive(&bars[B_PFULL]);
+      // K scaling after the mask: it overlaps P V(c) and S(c + 1) on the tensor cores
+      // ---- chunk-state operand (after the mask): K rows scaled by exp(G - g_s), hi in place, lo to klo ----
+      if (c + 1 < nch) {
+        if (c > 0) W(B_HFULL, (c - 1) & 1);   // H of the previous chunk has read klo
+        const float ks = row < n ? __expf(gend - g_row) : 0.f;
+        uint8_t* kt = stage(s) + kTile;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t off = sw128_off(row, part * 32 + j * 8);
+          const uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
+          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
+            split_pack(__low2float(pr) * ks, __high2float(pr) * ks, hi[e], lo[e]);
+          }
+          *reinterpret_cast<uint4*>(kt + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(klo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[B_KS]);
+      }
+
     }
-  } else {
+  } else if (warp < kPI2) {
     // ------------------------------------------------------------ group B
     const int half = (warp - kPB0) >> 2;   // which 32 of the 64 output columns
     const int j_dv = row & 63;             // merge: row of H^T (a d_v index) ...
@@ -963,21 +911,31 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[e] = 0.f;
       float gap = 0.f;
+      int cur0 = -1, cur1 = -1;  // readout chain being drained
 #pragma unroll
       for (int b = 0; b < kLevels; ++b) {
         if (!((c >> b) & 1)) continue;
-        const int rs = u & 1;
-        W(B_RFULL + rs, (u >> 1) & 1);
-        tc_fence_after();
+        if (b > cur1) {
+          if (cur1 >= 0) {
+            tc_fence_before();
+            mbar_arrive(&bars[B_REMPTY]);
+            ++u;
+          }
+          next_chain(c, b, cur0, cur1);
+          W(B_RFULL, u & 1);
+          tc_fence_after();
+        }
         const float w = lamv[b] * __expf(g_row + gap);
         float r0[32];
-        tmem_ld32(tmem + lane_off + kPColR + 64 * rs + 32 * half, r0);
+        tmem_ld32(tmem + lane_off + kPColR + 64 * (b - cur0) + 32 * half, r0);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars[B_REMPTY + rs]);
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = fmaf(w, r0[e], o[e]);
         gap += gtot[b];
+      }
+      if (cur1 >= 0) {
+        tc_fence_before();
+        mbar_arrive(&bars[B_REMPTY]);
         ++u;
       }
       // ---- Fenwick merge: level m = H + sum_{b<m} exp(decay after block b) S_b ----
@@ -992,12 +950,12 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         for (int b = 0; b < kLevels; ++b) {
           if (b < m) {
             const float f = __expf(acc);
-            const uint8_t* sl = slots + b * kSlot;
+            const uint8_t* sl = slots + b * 8192;
 #pragma unroll
             for (int qd = 0; qd < 2; ++qd) {
               const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
               const uint4 a4 = *reinterpret_cast<const uint4*>(sl + off);
-              const uint4 b4 = *reinterpret_cast<const uint4*>(sl + 8192 + off);
+              const uint4 b4 = *reinterpret_cast<const uint4*>(sl + kPLoOff + off);
               const uint32_t av[4] = {a4.x, a4.y, a4.z, a4.w};
               const uint32_t bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
@@ -1023,7 +981,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         }
         tc_fence_before();
         mbar_arrive(&bars[B_HEMPTY]);
-        uint8_t* dsl = slots + m * kSlot;
+        uint8_t* dsl = slots + m * 8192;
 #pragma unroll
         for (int qd = 0; qd < 2; ++qd) {
           uint32_t hi[4], lo[4];
@@ -1032,7 +990,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             split_pack(hv[8 * qd + 2 * e], hv[8 * qd + 2 * e + 1], hi[e], lo[e]);
           const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
           *reinterpret_cast<uint4*>(dsl + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(dsl + 8192 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(dsl + kPLoOff + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
         fence_proxy_async_smem();
 #pragma unroll
@@ -1058,6 +1016,54 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
       }
       mbar_arrive(&bars[B_GEMPTY + s]);
+    }
+  } else {
+    // ------------------------------------------------------------ inter-chunk MMA issuer
+    // Per chunk c: the readout chains of the set bits of c (they need the level states left
+    // by the merge after chunk c - 1), then H^T(c) if a merge follows (it needs the scaled K
+    // of chunk c).  Blocking waits, in chunk order: no barrier runs a phase ahead of this
+    // waiter, and a waiting issuer takes no issue slots from the math warps.
+    if (lane == 0) {
+      uint32_t u = 0;  // readout chains issued so far
+      for (int c = 0; c < nch; ++c) {
+        const int s = c & 1;
+        if (!W(B_FULL + s, (c >> 1) & 1)) break;
+        const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile, va = qa + 2 * kTile;
+        bool ok = true;
+        int cb0 = 0, cb1 = 0;
+        for (bool more = next_chain(c, 0, cb0, cb1); more; more = next_chain(c, cb1 + 1, cb0, cb1)) {
+          if ((c > 0 && !W(((c - 1) & 1) ? B_LV1 : B_LV, ((c - 1) >> 1) & 1)) ||
+              !W(B_REMPTY, (u & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t qd = kdesc(qa);
+          const uint64_t sd = kdesc(smem_u32(slots + cb0 * 8192));
+          const uint64_t sdl = kdesc(smem_u32(slots + kPLoOff + cb0 * 8192));
+          const uint32_t idr = idesc_bf16(128, 64 * (cb1 - cb0 + 1), 0, 0);
+#pragma unroll
+          for (int x = 0; x < kD / 16; ++x) mma_ss(tmem + kPColR, qd + 2 * x, sd + 2 * x, idr, x > 0);
+#pragma unroll
+          for (int x = 0; x < kD / 16; ++x) mma_ss(tmem + kPColR, qd + 2 * x, sdl + 2 * x, idr, 1);
+          mma_commit(&bars[B_RFULL]);
+          ++u;
+        }
+        if (!ok) break;
+        if (c + 1 < nch) {
+          if (!W(B_KS, c & 1) || !W(B_HEMPTY, (c & 1) ^ 1)) break;
+          tc_fence_after();
+          const uint64_t vd = mndesc_dup(va), kd = mndesc(ka), kld = mndesc(smem_u32(klo));
+#pragma unroll
+          for (int x = 0; x < kC / 16; ++x) mma_ss(tmem + kPColH, vd + 128 * x, kd + 128 * x, kIdescHT, x > 0);
+#pragma unroll
+          for (int x = 0; x < kC / 16; ++x) mma_ss(tmem + kPColH, vd + 128 * x, kld + 128 * x, kIdescHT, 1);
+          mma_commit(&bars[B_HFULL]);
+        }
+        mma_commit(&bars[B_EMPTY + s]);   // this issuer's reads of stage s are done
+      }
+      mma_commit(&bars[B_DRAIN2]);
+      mbar_wait(&bars[B_DRAIN2], 0, 200000000ull);
     }
   }
 
