@@ -83,12 +83,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi): packs (a, b) pairs of both parts.
+// x ~= hi + lo: hi = x with its low 16 bits cleared (a bf16 value, exact), lo = bf16(x - hi)
+// (x - hi is exact in fp32 and below 2^-7 |x|, so hi + lo carries ~16 significant bits).
+// Packs the (a, b) pairs of both parts; a goes to the low 16 bits.
 __device__ __forceinline__ void split_pack(float a, float b, uint32_t& hi, uint32_t& lo) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const float ah = __low2float(h), bh = __high2float(h);
-  hi = *reinterpret_cast<uint32_t*>(&h);
-  lo = pack_bf16(a - ah, b - bh);
+  const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u, ub = __float_as_uint(b) & 0xFFFF0000u;
+  hi = __byte_perm(ua, ub, 0x7632);  // high halves of a (low) and b (high)
+  lo = pack_bf16(a - __uint_as_float(ua), b - __uint_as_float(ub));
 }
 
 __device__ __forceinline__ float bf16_at(const uint8_t* p) {
@@ -518,26 +519,27 @@ constexpr uint32_t kPOffSlots = kPOffKlo + kTile;   // level hi parts, then leve
 constexpr uint32_t kPLoOff = kLevels * 8192;        // lo part of level b at + kPLoOff + b * 8 KB
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
 constexpr uint32_t kPOffLam = kPOffSlots + kLevels * kSlot;
-constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[2][128]
-constexpr uint32_t kPOffCj = kPOffG + 2 * kC * 4;
+constexpr int kPG = 3;                                         // g buffers
+constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[3][128]
+constexpr uint32_t kPOffCj = kPOffG + kPG * kC * 4;
 constexpr uint32_t kPOffScan = kPOffCj + kC * 4;
 constexpr uint32_t kPOffBar = kPOffScan + 64;
-constexpr int kPNumBars = 22;
+constexpr int kPNumBars = 24;
 constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
 constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
 
 constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (hi/lo)
 constexpr uint32_t kPColO = 128;   // P V accumulator
-constexpr uint32_t kPColH = 192;   // H^T = V^T K_s, rows duplicated in lanes 64..127
-constexpr uint32_t kPColR = 256;   // readout accumulator: up to four adjacent levels
-constexpr int kPSpan = 4;          // levels one readout chain covers (N = 64 per level)
+constexpr uint32_t kPColH = 192;   // V^T [K_hi | K_lo] (128 cols), rows duplicated in lanes 64..127
+constexpr uint32_t kPColR = 320;   // readout accumulator: up to three adjacent levels
+constexpr int kPSpan = 3;          // levels one readout chain covers (N = 64 per level)
 
-constexpr uint32_t kIdescHT = idesc_bf16(128, 64, 1, 1);  // V^T (M contiguous) x K_s (N contiguous)
+constexpr uint32_t kIdescHT = idesc_bf16(128, 128, 1, 1);  // V^T (M contiguous) x [K_hi | K_lo]
 
 enum : int {
   B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 5, B_SPEMPTY = 6, B_KS = 7, B_HFULL = 8,
   B_HEMPTY = 9, B_LV = 10, B_LV1 = 11, B_OFULL = 12, B_OEMPTY = 13, B_RFULL = 14,
-  B_REMPTY = 15, B_GREADY = 16, B_GEMPTY = 18, B_DRAIN = 20, B_DRAIN2 = 21
+  B_REMPTY = 15, B_GREADY = 16, B_GEMPTY = 19, B_DRAIN = 22, B_DRAIN2 = 23
 };
 
 // Wait on an mbarrier phase; returns false at once if the CTA has aborted, and aborts
@@ -549,9 +551,7 @@ __device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, uint32_t* 
   if (*ab) return false;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*ab) return false;
     if (globaltimer_ns() - t0 > 2000000000ull) {
       atomicOr(status, LLATTN_DEV_WAIT_TIMEOUT);
@@ -591,7 +591,8 @@ __device__ __forceinline__ uint64_t mndesc_dup(uint32_t saddr) { return sdesc_sw
 
 __global__ void __maxnreg__(96)
 tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-            const __grid_constant__ CUtensorMap tmv, const __nv_bfloat16* __restrict__ q,
+            const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+            const __nv_bfloat16* __restrict__ q,
             const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
             const float* __restrict__ log_a, const float* __restrict__ lam,
             float* __restrict__ out, int H, int T, int L, const int* __restrict__ cu,
@@ -628,10 +629,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   if (tid == 32) {
     for (int i = 0; i < kPNumBars; ++i) {
       uint32_t cnt = 1;  // TMA / tcgen05.commit arrivals
-      if (i == B_EMPTY || i == B_EMPTY + 1) cnt = 2;  // one commit from each MMA issuer
-      if (i == B_PFULL || i == B_KS || i == B_GREADY || i == B_GREADY + 1) cnt = kPNA;
-      if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY ||
-          i == B_REMPTY || i == B_GEMPTY || i == B_GEMPTY + 1)
+      if (i == B_EMPTY || i == B_EMPTY + 1) cnt = 3;  // both MMA issuers + the output store
+      if (i == B_PFULL || i == B_KS || (i >= B_GREADY && i < B_GREADY + kPG)) cnt = kPNA;
+      if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY || i == B_REMPTY ||
+          (i >= B_GEMPTY && i < B_GEMPTY + kPG))
         cnt = kPNB;
       mbar_init(&bars[i], cnt);
     }
@@ -726,16 +727,21 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
       if (part == 0) pf_la = okt ? __ldg(log_a + tok * H + h) : 0.f;
     };
-    prefetch(0);
-    for (int c = 0; c < nch; ++c) {
-      const int s = c & 1, kk = c >> 1;
+    // Decay scan of chunk c: g = inclusive cumsum of log a (warp shuffles + a cross-warp
+    // carry), the column factors cj and the pre-scaled lam table.  It runs after the mask of
+    // chunk c - 1 and before that chunk's K scaling, so it never waits behind the slowest
+    // K scaling warp.
+    float g_row = 0.f, g0 = 0.f, gend = 0.f;
+    bool factored = true;
+    auto decay_scan = [&](int c) {
+      const int gb = c % kPG, gk = c / kPG;  // g buffer and its use index
       const int n = min(kC, sp.len - c * kC);
       float pfc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) pfc[i] = pf[i];
       const float la = pf_la;
       if (c + 1 < nch) prefetch(c + 1);
-      W(B_GEMPTY + s, (kk & 1) ^ 1);   // group B is done with g[s] of chunk c - 2
+      W(B_GEMPTY + gb, (gk & 1) ^ 1);   // group B is done with g[gb] of chunk c - 3
       float x = la;
       if (part == 0) {
 #pragma unroll
@@ -746,20 +752,29 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         if (lane == 31) scan[sub] = x;
       }
       named_sync(1, kPNA);  // also: every mask read of the previous chunk is done
-#pragma unroll
-      for (int i = 0; i < 4; ++i) lamA[row * kPLamStride + part + 2 * i] = pfc[i];
       if (part == 0) {
         float off = 0.f;
         for (int w = 0; w < sub; ++w) off += scan[w];
-        gs[s * kC + row] = x + off;
+        gs[gb * kC + row] = x + off;
       }
       named_sync(1, kPNA);
-      const float g_row = gs[s * kC + row];
-      const float g0 = gs[s * kC];
-      const float gend = gs[s * kC + n - 1];
-      const bool factored = (g0 - gend) <= 80.f;
+      g_row = gs[gb * kC + row];
+      g0 = gs[gb * kC];
+      gend = gs[gb * kC + n - 1];
+      factored = (g0 - gend) <= 80.f;
       if (part == 0) cj[row] = factored ? __expf(g0 - g_row) : 0.f;
-      mbar_arrive(&bars[B_GREADY + s]);
+      // lam table of this row for levels 0..7, pre-multiplied by exp(g_i - g_0) when the
+      // decay factorises (the column factor exp(g_0 - g_j) is cj)
+      const float rsc = factored ? __expf(g_row - g0) : 1.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lamA[row * kPLamStride + part + 2 * i] = pfc[i] * rsc;
+      mbar_arrive(&bars[B_GREADY + gb]);
+    };
+    prefetch(0);
+    decay_scan(0);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1, kk = c >> 1;
+      const int n = min(kC, sp.len - c * kC);
       if (!is_full(c)) {
         // ragged last chunk: plain loads into the stage, rows past the end zero-filled
         W(B_EMPTY + s, (kk & 1) ^ 1);
@@ -784,27 +799,20 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       W(B_SFULL, c & 1);
       tc_fence_after();
       named_sync(1, kPNA);  // cj and the lam table are visible to the whole group
-      // ---- causal Fenwick mask on S -> P (hi/lo), one 32-key block at a time ----
+      // ---- causal Fenwick mask on S -> P (hi/lo), 16 keys at a time ----
+      // The two warps of a sub-partition take alternate 16-key groups, so each gets half of
+      // the diagonal block (per-element levels) and half of every off-diagonal block.
       const uint32_t spc = tmem + lane_off + kPColSP;
       const int rb = sub;
-      const float ri = factored ? __expf(g_row - g0) : 0.f;
       const float* lr = lamA + row * kPLamStride;
 #pragma unroll 1
-      for (int kb = part; kb < 4; kb += 2) {
+      for (int g16 = part; g16 < 8; g16 += 2) {  // keys 16*g16 .. 16*g16+15
+        const int kb = g16 >> 1;                // their 32-key block
+        uint32_t hi[8], lo[8];
         if (kb > rb) {
-          uint32_t z[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) z[e] = 0u;
-          tmem_st16(spc + 32 * kb, z);
-          tmem_st16(spc + 32 * kb + 16, z);
-          continue;
-        }
-        const float rsc = factored ? ri : 1.f;
-        // off-diagonal blocks have one Fenwick level; the diagonal block one per element
-        const float wblk = kb < rb ? lr[6 + (31 - __clz(rb ^ kb))] * rsc : 0.f;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          const int g16 = 2 * kb + hh;  // keys 16*g16 .. 16*g16+15
+          for (int e = 0; e < 8; ++e) { hi[e] = 0u; lo[e] = 0u; }
+        } else {
           float sv[16];
           tmem_ld16(spc + 16 * g16, sv);
           tmem_wait_ld();
@@ -819,43 +827,53 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) cw[e] = __expf(g_row - gs[s * kC + 16 * g16 + e]);
+            for (int e = 0; e < 16; ++e) cw[e] = __expf(g_row - gs[(c % kPG) * kC + 16 * g16 + e]);
           }
-          uint32_t hi[8], lo[8];
           if (kb < rb) {
+            // off-diagonal: one Fenwick level, 1 + msb(i ^ j) = 6 + msb(rb ^ kb)
+            const float wblk = lr[6 + (31 - __clz(rb ^ kb))];
 #pragma unroll
             for (int e = 0; e < 16; e += 2)
               split_pack(sv[e] * wblk * cw[e], sv[e + 1] * wblk * cw[e + 1], hi[e >> 1], lo[e >> 1]);
           } else {
+            // diagonal block: level 1 + msb(lane ^ jj) (0 when equal: clz(0) = 32), j <= i
+            const int j0 = 16 * (g16 & 1);
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
               float p[2];
 #pragma unroll
               for (int t2 = 0; t2 < 2; ++t2) {
-                const int jj = 16 * hh + e + t2;  // key index inside the 32-key block
-                const int lev = (jj == lane) ? 0 : (32 - __clz(jj ^ lane));
-                const float val = sv[e + t2] * (lr[lev] * rsc) * cw[e + t2];
+                const int jj = j0 + e + t2;
+                const float val = sv[e + t2] * lr[32 - __clz(jj ^ lane)] * cw[e + t2];
                 p[t2] = jj <= lane ? val : 0.f;
               }
               split_pack(p[0], p[1], hi[e >> 1], lo[e >> 1]);
             }
           }
-          tmem_st8(spc + 16 * g16, hi);
-          tmem_st8(spc + 16 * g16 + 8, lo);
         }
+        tmem_st8(spc + 16 * g16, hi);
+        tmem_st8(spc + 16 * g16 + 8, lo);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[B_PFULL]);
-      // K scaling after the mask: it overlaps P V(c) and S(c + 1) on the tensor cores
-      // ---- chunk-state operand (after the mask): K rows scaled by exp(G - g_s), hi in place, lo to klo ----
+      const float gend_c = gend;
+      if (c + 1 < nch) decay_scan(c + 1);
+      // ---- chunk-state operand: K rows scaled by exp(G - g_s), hi in place, lo to klo ----
+      // (after the mask, overlapping P V(c) and S(c + 1) on the tensor cores).  The causal
+      // mask loads sub-partitions 0..3 in the ratio 1:2:3:4, so the K rows are dealt out the
+      // other way round: 48, 40, 24 and 16 rows to the two warps of sub-partitions 0..3.
       if (c + 1 < nch) {
         if (c > 0) W(B_HFULL, (c - 1) & 1);   // H of the previous chunk has read klo
-        const float ks = row < n ? __expf(gend - g_row) : 0.f;
         uint8_t* kt = stage(s) + kTile;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t off = sw128_off(row, part * 32 + j * 8);
+        const int r0 = sub == 0 ? 0 : (sub == 1 ? 48 : (sub == 2 ? 88 : 112));
+        const int nrows = sub == 0 ? 48 : (sub == 1 ? 40 : (sub == 2 ? 24 : 16));
+        const int t64 = part * 32 + lane;
+#pragma unroll 1
+        for (int unit = t64; unit < nrows * 8; unit += 64) {
+          const int kr = r0 + (unit >> 3);
+          const float ks = kr < n ? __expf(gend_c - gs[(c % kPG) * kC + kr]) : 0.f;
+          const uint32_t off = sw128_off(kr, (unit & 7) * 8);
           const uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
           const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t hi[4], lo[4];
@@ -897,9 +915,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     for (int c = 0; c < nch; ++c) {
       const int s = c & 1, kk = c >> 1;
       const int n = min(kC, sp.len - c * kC);
-      W(B_GREADY + s, kk & 1);
-      const float g_row = gs[s * kC + row];
-      const float gend = gs[s * kC + n - 1];
+      W(B_GREADY + c % kPG, (c / kPG) & 1);
+      const float g_row = gs[(c % kPG) * kC + row];
+      const float gend = gs[(c % kPG) * kC + n - 1];
       float lamv[kLevels];
 #pragma unroll
       for (int b = 0; b < kLevels; ++b) lamv[b] = pl[b];
@@ -973,11 +991,13 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         W(B_HFULL, c & 1);
         tc_fence_after();
         {
-          float t16[16];
-          tmem_ld16(tmem + lane_off + kPColH + 32 * (row >> 6) + 16 * half, t16);
+          // H^T = V^T K_hi (columns 0..63) + V^T K_lo (64..127); this thread's 16 d_k columns
+          float t16[16], u16[16];
+          tmem_ld16(tmem + lane_off + kPColH + dk0, t16);
+          tmem_ld16(tmem + lane_off + kPColH + 64 + dk0, u16);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) hv[e] += t16[e];
+          for (int e = 0; e < 16; ++e) hv[e] += t16[e] + u16[e];
         }
         tc_fence_before();
         mbar_arrive(&bars[B_HEMPTY]);
@@ -1009,13 +1029,36 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
       tc_fence_before();
       mbar_arrive(&bars[B_OEMPTY]);
-      if (row < n) {
-        float* dst = out + ((sp.start + (long long)c * kC + row) * H + h) * kD + 32 * half;
+      if (n == kC) {
+        // Whole chunk: stage the 128 x 64 fp32 tile in the Q (columns 0..31) and K (32..63)
+        // tiles of this stage -- every reader of them is done by now -- in the 128-byte
+        // swizzle, and let TMA write it out; row-per-thread global stores would touch one
+        // cache line per lane.
+        uint8_t* stg = stage(s) + half * kTile;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        for (int qd = 0; qd < 8; ++qd)
+          *reinterpret_cast<float4*>(stg + row * 128 + ((qd ^ (row & 7)) << 4)) =
+              make_float4(o[4 * qd], o[4 * qd + 1], o[4 * qd + 2], o[4 * qd + 3]);
+        fence_proxy_async_smem();
+        named_sync(2, kPNB);
+        if (warp == kPB0 && lane == 0) {
+          const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
+          tma_store_3d(&tmo, stage(s), 0, h, tok0);
+          tma_store_3d(&tmo, stage(s) + kTile, 32, h, tok0);
+          bulk_commit();
+          bulk_wait_read();
+          mbar_arrive(&bars[B_EMPTY + s]);  // the stage may be refilled
+        }
+      } else {
+        if (row < n) {
+          float* dst = out + ((sp.start + (long long)c * kC + row) * H + h) * kD + 32 * half;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        }
+        if (warp == kPB0 && lane == 0) mbar_arrive(&bars[B_EMPTY + s]);
       }
-      mbar_arrive(&bars[B_GEMPTY + s]);
+      mbar_arrive(&bars[B_GEMPTY + c % kPG]);
     }
   } else {
     // ------------------------------------------------------------ inter-chunk MMA issuer
@@ -1053,11 +1096,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         if (c + 1 < nch) {
           if (!W(B_KS, c & 1) || !W(B_HEMPTY, (c & 1) ^ 1)) break;
           tc_fence_after();
-          const uint64_t vd = mndesc_dup(va), kd = mndesc(ka), kld = mndesc(smem_u32(klo));
+          // B = [K_hi | K_lo]: two 64-wide N groups, the second at the klo tile (LBO)
+          const uint64_t vd = mndesc_dup(va);
+          const uint64_t kd = sdesc_sw128(ka, smem_u32(klo) - ka, 1024);
 #pragma unroll
           for (int x = 0; x < kC / 16; ++x) mma_ss(tmem + kPColH, vd + 128 * x, kd + 128 * x, kIdescHT, x > 0);
-#pragma unroll
-          for (int x = 0; x < kC / 16; ++x) mma_ss(tmem + kPColH, vd + 128 * x, kld + 128 * x, kIdescHT, 1);
           mma_commit(&bars[B_HFULL]);
         }
         mma_commit(&bars[B_EMPTY + s]);   // this issuer's reads of stage s are done
@@ -1067,6 +1110,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     }
   }
 
+  if (warp == kPB0 && lane == 0) bulk_wait_all();  // output tiles written
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1110,6 +1154,20 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int H, long long tokens) 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// out [tokens, H, 64] fp32 as {64, H, tokens}; box {32, 1, 128} (128 B rows), 128 B swizzle.
+cudaError_t make_out_map(CUtensorMap* m, void* base, int H, long long tokens) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {kD, (cuuint64_t)H, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {kD * 4, (cuuint64_t)H * kD * 4};
+  const cuuint32_t box[3] = {32, 1, kC};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T) {
@@ -1129,6 +1187,8 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
   if ((e = make_map(&mq, p.q, p.H, tokens)) != cudaSuccess) return e;
   if ((e = make_map(&mk, p.k, p.H, tokens)) != cudaSuccess) return e;
   if ((e = make_map(&mv, p.v, p.H, tokens)) != cudaSuccess) return e;
+  CUtensorMap mo;
+  if ((e = make_out_map(&mo, p.out, p.H, tokens)) != cudaSuccess) return e;
   static bool attr_set = false;
   if (!attr_set) {
     if ((e = cudaFuncSetAttribute(tc_fwd_serial, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1148,7 +1208,7 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
     tc_fwd_serial<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, q, k, v, p.log_a, p.lam, p.out,
                                                       p.H, p.T, p.L, p.cu_seqlens, p.status);
   else
-    tc_fwd_pipe<<<grid, kPThreads, kPSmemBytes, st>>>(mq, mk, mv, q, k, v, p.log_a, p.lam, p.out,
+    tc_fwd_pipe<<<grid, kPThreads, kPSmemBytes, st>>>(mq, mk, mv, mo, q, k, v, p.log_a, p.lam, p.out,
                                                       p.H, p.T, p.L, p.cu_seqlens, p.status);
   main_kernel_end(st);
   count_launch();
