@@ -219,6 +219,22 @@ def run_reference(args, w, rank, world):
     return line
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest per-rank value over all ranks (the slowest rank sets the step time);
+    `dist` is torch.distributed or None for a single process."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: per-GPU work fixed as N grows)."""
+    return seed + rank
+
+
 def workload_config(w, chunk, path):
     cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "L": w.L,
            "inputs": f"{w.dtype} q/k/v, f32 log_a/lam, f32 out",
@@ -246,7 +262,7 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     binding.lib()
-    inp = I.make_inputs(w, seed=args.seed + rank)
+    inp = I.make_inputs(w, seed=rank_seed(args.seed, rank))
     dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
     q = torch.from_numpy(inp.q).to(dev).to(dt)
     k = torch.from_numpy(inp.k).to(dev).to(dt)
@@ -300,12 +316,8 @@ def run_ours(args, w, rank, world, local_rank):
         dist.barrier()
     binding.profile(False)
     clk = clocks.stop()
-    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     main_ms, main_n, launches = binding.profile_read(reset=True)
-    if dist:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     status = binding.device_status(clear=True)
     if status:
         raise RuntimeError(f"device status flags {status:#x} after the timed region")
@@ -374,15 +386,14 @@ def run_ours(args, w, rank, world, local_rank):
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
+        # device-timed on the stream the host entry point copies and computes on; each call
+        # synchronises that stream, so host-side gaps between calls are inside the bracket too
+        e0.record(stream)
         for _ in range(n_e2e):
             e2e_step()
+        e1.record(stream)
         torch.cuda.synchronize()
-        e2e_s = (time.perf_counter() - t0) / n_e2e
-        if dist:
-            t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_s = float(t.item())
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1000.0 / n_e2e, dist, dev)
         ref_host = hout.numpy()
         if not np.isfinite(ref_host).all():
             raise RuntimeError("non-finite output through the host entry point")

@@ -500,8 +500,8 @@ tc_fwd_serial(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
 //   warp 18       MMA issuer for the inter-chunk part (H^T, level readouts)
 //   warps 2..9    group A      (decay scan, K scaling for the chunk state, causal mask -> P)
 //   warps 10..17  group B      (Fenwick merge of the chunk state, epilogue and store)
-// TMEM holds S/P, the P V accumulator, H^T and four level-readout accumulators, so a
-// chunk's readouts (up to four levels at once) are in flight together.
+// TMEM holds S/P, the P V accumulator, H^T (twice, for hi and lo K) and one readout
+// accumulator spanning up to three adjacent levels, so one MMA chain reads them together.
 // P overwrites S in place, 16 keys at a time: the 16 fp32 columns of keys 16g..16g+15
 // become 8 columns of bf16 pairs (hi) followed by 8 (lo), so no thread ever writes
 // columns that it or another thread has still to read.

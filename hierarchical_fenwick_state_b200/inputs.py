@@ -205,6 +205,33 @@ def make_inputs(w: Workload, seed: int = 0, *, log_a_mode: str = "dist",
                   B=B, H=H, T=w.T, dk=dk, dv=dv, dtype=w.dtype)
 
 
+def make_patterned(T: int, *, H: int = 1, dk: int = 64, dv: int = 64, log_a: float = 0.0,
+                   dtype: str = "bf16") -> Inputs:
+    """Deterministic small-integer inputs given by closed forms, for the golden fixtures.
+
+    q[t,h,i] = ((3t + 5i + h) mod 7) - 3,   k[t,h,i] = ((5t + 3i + 2h + 1) mod 7) - 3,
+    v[t,h,j] = ((2t + 7j + h + 3) mod 5) - 2,
+    log_a[t,h] = log_a (one constant),      lam[t,h,l] = 1 + ((t + 3l + h) mod 4) / 4.
+    Every value is exact in bf16 and fp32 (log_a too when it is a short binary fraction), so
+    the outputs can be known exactly and every dtype sees the same numbers.  One dense
+    sequence (B = 1).
+    """
+    t = np.arange(T)[:, None, None]
+    h = np.arange(H)[None, :, None]
+    i = np.arange(dk)[None, None, :]
+    j = np.arange(dv)[None, None, :]
+    L = num_levels(T)
+    lv = np.arange(L)[None, None, :]
+    q = ((3 * t + 5 * i + h) % 7 - 3).astype(np.float32)[None]
+    k = ((5 * t + 3 * i + 2 * h + 1) % 7 - 3).astype(np.float32)[None]
+    v = ((2 * t + 7 * j + h + 3) % 5 - 2).astype(np.float32)[None]
+    la = np.full((1, T, H), log_a, dtype=np.float32)
+    lam = (1.0 + ((t + 3 * lv + h) % 4) / 4.0).astype(np.float32)[None]
+    return Inputs(q=np.ascontiguousarray(q), k=np.ascontiguousarray(k),
+                  v=np.ascontiguousarray(v), log_a=la, lam=np.ascontiguousarray(lam),
+                  cu_seqlens=None, B=1, H=H, T=T, dk=dk, dv=dv, dtype=dtype)
+
+
 def shrink(w: Workload, *, B: Optional[int] = None, H: Optional[int] = None,
            T: Optional[int] = None, len_lo: Optional[int] = None,
            len_hi: Optional[int] = None, name: Optional[str] = None) -> Workload:

@@ -152,3 +152,21 @@ def test_full_size_sampled(name):
     assert np.isfinite(got).all()
     err = O.rel_max_err(sel, ref)
     assert err <= TOL[inp.dtype], f"{name}: sampled rel max err {err:.3e}"
+
+
+# ------------------------------------------------------------------------------------------------
+# Golden fixtures: closed-form integer inputs whose outputs are stored in tests/golden/
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name,decay", [("patterned_nodecay_T300", 0.0),
+                                        ("patterned_decay8_T300", -0.125)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_golden_fixtures(name, decay, dtype):
+    from test_golden import load
+    inp = I.make_patterned(300, log_a=decay, dtype=dtype)
+    rows = load(name)
+    want = np.array([o for _, _, o in rows])
+    for path in _paths_for(inp):
+        got = run(inp, path=path).reshape(300, inp.H, inp.dv)
+        sel = np.array([got[t, 0, j] for t, j, _ in rows])
+        err = O.rel_max_err(sel, want)
+        assert err <= TOL[dtype], f"{path}: rel max err {err:.3e}"
