@@ -22,7 +22,10 @@ EXPORTS = (
     "llattn_abi_version", "llattn_status_str", "llattn_num_levels", "llattn_fwd",
     "llattn_fwd_f32", "llattn_workspace_bytes", "llattn_fwd_ex", "llattn_device_status",
     "llattn_last_cuda_error", "llattn_fwd_host", "llattn_profile", "llattn_profile_read",
+    "llattn_fwd_noalloc",
 )
+
+NOALLOC_SCRATCH_BYTES = 32 << 20  # LLATTN_NOALLOC_SCRATCH_BYTES
 
 _lib = None
 
@@ -65,6 +68,8 @@ def lib():
     L.llattn_last_cuda_error.restype = i
     L.llattn_fwd_host.restype = i
     L.llattn_fwd_host.argtypes = [i, vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_fwd_noalloc.restype = i
+    L.llattn_fwd_noalloc.argtypes = [i, vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
     L.llattn_profile.restype = i
     L.llattn_profile.argtypes = [i]
     L.llattn_profile_read.restype = i
@@ -181,6 +186,21 @@ def fwd_host(in_dtype: int, q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlen
                                int(B), int(H), int(T), int(dk), int(dv), ptr(cu_seqlens),
                                _stream_handle(stream) if stream is not None else None)
     _check(st, "llattn_fwd_host")
+    return out
+
+
+def fwd_noalloc(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None, stream=None):
+    """Direct call of llattn_fwd_noalloc on raw device tensors (bf16 or fp32 q/k/v):
+    the forward with no device allocation, scratch from the library's fixed array."""
+    in_dtype = BF16 if str(q.dtype) == "torch.bfloat16" else F32
+    st = lib().llattn_fwd_noalloc(in_dtype, ctypes.c_void_p(q.data_ptr()),
+                                  ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+                                  ctypes.c_void_p(log_a.data_ptr()),
+                                  ctypes.c_void_p(lam.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                  int(B), int(H), int(T), int(dk), int(dv),
+                                  ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None
+                                  else None, _stream_handle(stream))
+    _check(st, "llattn_fwd_noalloc")
     return out
 
 

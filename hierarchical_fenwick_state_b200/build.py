@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["llattn_api.cu", "llattn_simt.cu", "llattn_tc.cu"]
+SOURCES = ["llattn_api.cu", "llattn_simt.cu", "llattn_tc.cu", "llattn_noalloc.cu"]
 HEADERS = ["llattn_internal.h", "llattn_common.cuh", "llattn_tc_ptx.cuh"]
 LIB = os.path.join(HERE, "libllattn.so")
 BUILD_DIR = os.path.join(ROOT, "_build")

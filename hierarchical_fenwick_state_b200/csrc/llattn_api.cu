@@ -250,6 +250,8 @@ const char* llattn_status_str(llattn_status s) {
     case LLATTN_ERR_TIMEOUT: return "device-side wait timed out";
     case LLATTN_ERR_WORKSPACE: return "workspace too small or misaligned";
     case LLATTN_ERR_UNSUPPORTED: return "no kernel for this configuration";
+    case LLATTN_ERR_NOALLOC_LIMIT:
+      return "problem needs more scratch than llattn_fwd_noalloc's fixed array holds";
   }
   return "unknown status";
 }
@@ -294,6 +296,26 @@ llattn_status llattn_fwd_ex(int in_dtype, int path, int chunk, const void* q, co
                             void* workspace, size_t workspace_bytes, void* stream) {
   return forward(in_dtype, path, chunk, q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens,
                  workspace, workspace_bytes, stream);
+}
+
+llattn_status llattn_fwd_noalloc(int in_dtype, const void* q, const void* k, const void* v,
+                                 const float* log_a, const float* lam, float* out, int B, int H,
+                                 int T, int dk, int dv, const int* cu_seqlens, void* stream) {
+  // Size check first: it needs no device, and a rejected call touches nothing.
+  size_t need = 0;
+  llattn_status s = llattn_workspace_bytes(in_dtype, LLATTN_PATH_SIMT, 0, B, H, T, dk, dv,
+                                           cu_seqlens != nullptr, &need);
+  if (s != LLATTN_OK) return s;
+  if (need > LLATTN_NOALLOC_SCRATCH_BYTES) return LLATTN_ERR_NOALLOC_LIMIT;
+  if (need == 0)  // empty problem: nothing is launched and no scratch is used
+    return forward(in_dtype, LLATTN_PATH_SIMT, 0, q, k, v, log_a, lam, out, B, H, T, dk, dv,
+                   cu_seqlens, nullptr, 0, stream);
+  void* scratch = nullptr;
+  cudaError_t e = llattn::noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // A caller-supplied workspace never reaches the library's allocator.
+  return forward(in_dtype, LLATTN_PATH_SIMT, 0, q, k, v, log_a, lam, out, B, H, T, dk, dv,
+                 cu_seqlens, scratch, LLATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 llattn_status llattn_device_status(unsigned int* flags, int clear) {

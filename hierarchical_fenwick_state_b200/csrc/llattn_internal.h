@@ -37,6 +37,10 @@ cudaError_t simt_forward(const Problem& p, int chunk, void* ws, cudaStream_t st)
 cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, bool serial);
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T);
 
+// Device address of the fixed scratch array behind llattn_fwd_noalloc on the
+// current device (looked up on the first call per device, then cached).
+cudaError_t noalloc_scratch(void** ptr);
+
 // Number of chunk-level Fenwick blocks kept per (sequence, head) for Nc chunks,
 // and the offset of level b's blocks: level b holds blocks (b, j) for even j,
 // i.e. ((Nc - 1) >> (b + 1)) + 1 of them (only levels with 2^b < Nc).

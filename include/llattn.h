@@ -69,7 +69,8 @@ typedef enum {
   LLATTN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
   LLATTN_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out (see llattn_device_status) */
   LLATTN_ERR_WORKSPACE = 7,   /* caller workspace too small or misaligned */
-  LLATTN_ERR_UNSUPPORTED = 8  /* valid request this build has no kernel for */
+  LLATTN_ERR_UNSUPPORTED = 8, /* valid request this build has no kernel for */
+  LLATTN_ERR_NOALLOC_LIMIT = 9 /* llattn_fwd_noalloc: problem too big for its fixed scratch */
 } llattn_status;
 
 /* Input element types for llattn_fwd_ex. */
@@ -167,6 +168,54 @@ LLATTN_API llattn_status llattn_device_status(unsigned int* flags, int clear);
 LLATTN_API llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const void* v,
                               const float* log_a, const float* lam, float* out, int B, int H,
                               int T, int dk, int dv, const int* cu_seqlens, void* stream);
+
+/*
+ * llattn_fwd_noalloc - the forward for callers that must not have a library
+ * allocate device memory on their behalf.  Typical cases: an application whose
+ * own allocator reserves nearly all of the GPU's memory up front, where a
+ * cudaMalloc issued here would fail or eat into memory that allocator has
+ * promised elsewhere; a service that must know its whole device footprint before
+ * it takes traffic; and latency-bound code, because the buffer behind llattn_fwd
+ * grows by cudaFree + cudaMalloc, and cudaFree waits for the whole device,
+ * stalling every stream of the process.  This entry point has no counterpart in
+ * the log-linear attention papers; it is packaging around the same operation.
+ *
+ * It computes what llattn_fwd_ex computes with path LLATTN_PATH_SIMT and the
+ * default chunk (CUDA cores, fp32 arithmetic; in_dtype LLATTN_F32 or
+ * LLATTN_BF16), and takes its inter-chunk scratch from one array of
+ * LLATTN_NOALLOC_SCRATCH_BYTES (32 MiB) per device that is part of the library's
+ * device code itself.  Arguments, layouts, ownership, the device status word and
+ * the other error codes are those of llattn_fwd_ex.
+ *
+ * Size limit.  The problem's scratch, as reported by llattn_workspace_bytes(
+ * in_dtype, LLATTN_PATH_SIMT, 0, B, H, T, dk, dv, cu_seqlens != NULL, &n), must
+ * not exceed LLATTN_NOALLOC_SCRATCH_BYTES.  Larger problems return
+ * LLATTN_ERR_NOALLOC_LIMIT (after the shape and dtype checks, before the pointer
+ * checks) without making any CUDA call.  For scale: B=2, H=16, T=2048, dk=dv=64 needs 31.5 MiB and fits;
+ * B=4, H=32, T=8192 does not.
+ *
+ * Setup.  The first call on a device that has work to do looks up the array's
+ * address there (cudaGetSymbolAddress, with that device current), keeps it, and
+ * returns LLATTN_ERR_CUDA if the lookup fails.  That first call should come
+ * before any stream capture.  Later calls only launch kernels.
+ *
+ * Zeroing.  Each call writes every scratch entry it reads before reading it, so
+ * no part of the array has to start at zero and nothing is cleared between calls.
+ * The device status word keeps its meaning (sticky until llattn_device_status
+ * clears it).
+ *
+ * Concurrency.  There is one array per device, shared by every caller in the
+ * process.  Calls whose kernels can overlap on the GPU (on different streams, or
+ * from host threads that do not order their streams) race on it and can corrupt
+ * one another's output.  Calls on one stream run one after another and are safe.
+ * With launch recording on (llattn_profile(1)) the library may create CUDA events
+ * for its timing pairs; it is off by default.
+ */
+#define LLATTN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+LLATTN_API llattn_status llattn_fwd_noalloc(int in_dtype, const void* q, const void* k,
+                                            const void* v, const float* log_a, const float* lam,
+                                            float* out, int B, int H, int T, int dk, int dv,
+                                            const int* cu_seqlens, void* stream);
 
 /*
  * Launch accounting, for benchmarks.  llattn_profile(1) starts recording a pair
