@@ -522,9 +522,12 @@ constexpr uint32_t kPOffLam = kPOffSlots + kLevels * kSlot;
 constexpr int kPG = 3;                                         // g buffers
 constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[3][128]
 constexpr uint32_t kPOffCj = kPOffG + kPG * kC * 4;
-constexpr uint32_t kPOffScan = kPOffCj + kC * 4;
+// lam of the inter-chunk levels 1+log2 C+b (b < kLevels) times exp(g_i), per row: group A
+// writes it with the decay scan, group B reads it for the readout weights (g buffers' ring)
+constexpr uint32_t kPOffLamB = kPOffCj + kC * 4;
+constexpr uint32_t kPOffScan = kPOffLamB + kPG * kC * kLevels * 4;
 constexpr uint32_t kPOffBar = kPOffScan + 64;
-constexpr int kPNumBars = 24;
+constexpr int kPNumBars = 27;
 constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
 constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
 
@@ -539,7 +542,8 @@ constexpr uint32_t kIdescHT = idesc_bf16(128, 128, 1, 1);  // V^T (M contiguous)
 enum : int {
   B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 5, B_SPEMPTY = 6, B_KS = 7, B_HFULL = 8,
   B_HEMPTY = 9, B_LV = 10, B_LV1 = 11, B_OFULL = 12, B_OEMPTY = 13, B_RFULL = 14,
-  B_REMPTY = 15, B_GREADY = 16, B_GEMPTY = 19, B_DRAIN = 22, B_DRAIN2 = 23
+  B_REMPTY = 15, B_GREADY = 16, B_GEMPTY = 19, B_DRAIN = 22, B_DRAIN2 = 23, B_OSTAGED = 24,
+  B_FREE = 26
 };
 
 // Wait on an mbarrier phase; returns false at once if the CTA has aborted, and aborts
@@ -617,6 +621,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   float* lamA = reinterpret_cast<float*>(sm + kPOffLam);
   float* gs = reinterpret_cast<float*>(sm + kPOffG);
   float* cj = reinterpret_cast<float*>(sm + kPOffCj);
+  float* lamB = reinterpret_cast<float*>(sm + kPOffLamB);
   float* scan = reinterpret_cast<float*>(sm + kPOffScan);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kPOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kPOffMisc);  // [0] TMEM base, [1] abort
@@ -629,10 +634,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   if (tid == 32) {
     for (int i = 0; i < kPNumBars; ++i) {
       uint32_t cnt = 1;  // TMA / tcgen05.commit arrivals
-      if (i == B_EMPTY || i == B_EMPTY + 1) cnt = 3;  // both MMA issuers + the output store
+      if (i == B_EMPTY || i == B_EMPTY + 1) cnt = 2;  // both MMA issuers
       if (i == B_PFULL || i == B_KS || (i >= B_GREADY && i < B_GREADY + kPG)) cnt = kPNA;
       if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY || i == B_REMPTY ||
-          (i >= B_GEMPTY && i < B_GEMPTY + kPG))
+          (i >= B_GEMPTY && i < B_GEMPTY + kPG) || i == B_OSTAGED || i == B_OSTAGED + 1)
         cnt = kPNB;
       mbar_init(&bars[i], cnt);
     }
@@ -651,18 +656,44 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Loads Q, K, V of chunk c into stage c % 2 once that stage is free: both MMA issuers are
+    // done with chunk c - 2, whose output tile group B staged there, and this thread has
+    // stored that tile (TMA store, waited until its shared-memory reads are done).  Doing the
+    // store here keeps its wait out of group B's chunk loop.  A ragged last chunk is loaded
+    // by group A with plain loads; B_FREE tells it the stage is free.
     if (lane == 0) {
       int last0 = -1, last1 = -1;
-      for (int c = 0; c < nch && is_full(c); ++c) {
+      bool ok = true;
+      auto store_out = [&](int cc) {
+        if (!W(B_OSTAGED + (cc & 1), (cc >> 1) & 1)) return false;
+        if (is_full(cc)) {
+          const int tok0 = static_cast<int>(sp.start + (long long)cc * kC);
+          tma_store_3d(&tmo, stage(cc & 1), 0, h, tok0);
+          tma_store_3d(&tmo, stage(cc & 1) + kTile, 32, h, tok0);
+          bulk_commit();
+          bulk_wait_read();
+        }
+        return true;
+      };
+      for (int c = 0; c < nch; ++c) {
         const int s = c & 1, kk = c >> 1;
-        if (!W(B_EMPTY + s, (kk & 1) ^ 1)) break;
-        const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
-        mbar_arrive_expect_tx(&bars[B_FULL + s], 3 * kTile);
-        tma_load_3d(stage(s), &tmq, &bars[B_FULL + s], 0, h, tok0);
-        tma_load_3d(stage(s) + kTile, &tmk, &bars[B_FULL + s], 0, h, tok0);
-        tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[B_FULL + s], 0, h, tok0);
-        if (s == 0) last0 = c; else last1 = c;
+        if (c >= 2 && (!W(B_EMPTY + s, (kk & 1) ^ 1) || !store_out(c - 2))) {
+          ok = false;
+          break;
+        }
+        if (is_full(c)) {
+          const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
+          mbar_arrive_expect_tx(&bars[B_FULL + s], 3 * kTile);
+          tma_load_3d(stage(s), &tmq, &bars[B_FULL + s], 0, h, tok0);
+          tma_load_3d(stage(s) + kTile, &tmk, &bars[B_FULL + s], 0, h, tok0);
+          tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[B_FULL + s], 0, h, tok0);
+          if (s == 0) last0 = c; else last1 = c;
+        } else {
+          mbar_arrive(&bars[B_FREE]);
+        }
       }
+      for (int cc = nch > 2 ? nch - 2 : 0; ok && cc < nch; ++cc) ok = store_out(cc);
+      bulk_wait_all();  // output tiles written
       if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) {
         // an aborted CTA still lets its own copies land before it exits
         if (last0 >= 0) mbar_wait(&bars[B_FULL + 0], (last0 >> 1) & 1, 200000000ull);
@@ -713,7 +744,8 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     // ------------------------------------------------------------ group A
     const int wa = warp - kPA0;     // 0..7
     const int part = wa >> 2;       // column blocks part, part + 2; K columns 32*part..
-    float pf[4];
+    constexpr int kNP = (kLogC + 1 + kLevels) / 2;   // lam levels per thread: 0..13 over 2 parts
+    float pf[kNP];
     float pf_la = 0.f;
     auto prefetch = [&](int c) {
       const int t = c * kC + row;
@@ -721,7 +753,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       const long long tok = sp.start + t;
       const float* lr = lam + (tok * H + h) * L;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kNP; ++i) {
         const int l = part + 2 * i;
         pf[i] = (okt && l < L) ? __ldg(lr + l) : 0.f;
       }
@@ -736,9 +768,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     auto decay_scan = [&](int c) {
       const int gb = c % kPG, gk = c / kPG;  // g buffer and its use index
       const int n = min(kC, sp.len - c * kC);
-      float pfc[4];
+      float pfc[kNP];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pfc[i] = pf[i];
+      for (int i = 0; i < kNP; ++i) pfc[i] = pf[i];
       const float la = pf_la;
       if (c + 1 < nch) prefetch(c + 1);
       W(B_GEMPTY + gb, (gk & 1) ^ 1);   // group B is done with g[gb] of chunk c - 3
@@ -768,6 +800,12 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       const float rsc = factored ? __expf(g_row - g0) : 1.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) lamA[row * kPLamStride + part + 2 * i] = pfc[i] * rsc;
+      // inter-chunk levels for group B's readout weights, with the row's decay from the chunk
+      // start (g_row <= 0, so the factor stays finite)
+      const float eg = __expf(g_row);
+#pragma unroll
+      for (int i = 4; i < kNP; ++i)
+        lamB[(gb * kC + row) * kLevels + part + 2 * i - (kLogC + 1)] = pfc[i] * eg;
       mbar_arrive(&bars[B_GREADY + gb]);
     };
     prefetch(0);
@@ -776,8 +814,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       const int s = c & 1, kk = c >> 1;
       const int n = min(kC, sp.len - c * kC);
       if (!is_full(c)) {
-        // ragged last chunk: plain loads into the stage, rows past the end zero-filled
-        W(B_EMPTY + s, (kk & 1) ^ 1);
+        // ragged last chunk: plain loads into the stage, rows past the end zero-filled, once
+        // the producer has stored the output tile of chunk c - 2 from it
+        W(B_FREE, 0);
         const long long tok0 = sp.start + (long long)c * kC;
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
@@ -895,19 +934,6 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     const int half = (warp - kPB0) >> 2;   // which 32 of the 64 output columns
     const int j_dv = row & 63;             // merge: row of H^T (a d_v index) ...
     const int dk0 = 32 * (row >> 6) + 16 * half;  // ... and the 16 d_k columns it merges
-    float pl[kLevels];
-    auto prefetch = [&](int c) {
-      const int t = c * kC + row;
-      const bool okt = t < sp.len;
-      const long long tok = sp.start + t;
-      const float* lr = lam + (tok * H + h) * L;
-#pragma unroll
-      for (int b = 0; b < kLevels; ++b) {
-        const int l = 1 + kLogC + b;
-        pl[b] = (okt && l < L && ((c >> b) & 1)) ? __ldg(lr + l) : 0.f;
-      }
-    };
-    prefetch(0);
     float gtot[kLevels];
 #pragma unroll
     for (int b = 0; b < kLevels; ++b) gtot[b] = 0.f;
@@ -916,18 +942,23 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       const int s = c & 1, kk = c >> 1;
       const int n = min(kC, sp.len - c * kC);
       W(B_GREADY + c % kPG, (c / kPG) & 1);
-      const float g_row = gs[(c % kPG) * kC + row];
       const float gend = gs[(c % kPG) * kC + n - 1];
-      float lamv[kLevels];
+      const float* lamv = lamB + ((c % kPG) * kC + row) * kLevels;
+      // ---- epilogue: o = P V + sum_b lam[., 1+log2 C+b] exp(g + gap_b) R_b ----
+      // P V first: it seeds the accumulator and frees the P V columns for chunk c + 1 at once.
+      // Pairs of columns go through the packed f32x2 pipe.
+      float2 o2[16];
+      W(B_OFULL, c & 1);
+      tc_fence_after();
+      {
+        float r0[32];
+        tmem_ld32(tmem + lane_off + kPColO + 32 * half, r0);
+        tmem_wait_ld();
 #pragma unroll
-      for (int b = 0; b < kLevels; ++b) lamv[b] = pl[b];
-      if (c + 1 < nch) prefetch(c + 1);
-      // ---- epilogue: o = sum_b lam[., 1+log2 C+b] exp(g + gap_b) R_b + P V ----
-      // The readouts are drained first: the MMA warp issues them before P V and may be
-      // waiting for a free readout accumulator.
-      float o[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        for (int e = 0; e < 16; ++e) o2[e] = make_float2(r0[2 * e], r0[2 * e + 1]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_OEMPTY]);
       float gap = 0.f;
       int cur0 = -1, cur1 = -1;  // readout chain being drained
 #pragma unroll
@@ -943,12 +974,13 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           W(B_RFULL, u & 1);
           tc_fence_after();
         }
-        const float w = lamv[b] * __expf(g_row + gap);
+        const float w = lamv[b] * __expf(gap);
+        const float2 w2 = make_float2(w, w);
         float r0[32];
         tmem_ld32(tmem + lane_off + kPColR + 64 * (b - cur0) + 32 * half, r0);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = fmaf(w, r0[e], o[e]);
+        for (int e = 0; e < 16; ++e) o2[e] = __ffma2_rn(w2, make_float2(r0[2 * e], r0[2 * e + 1]), o2[e]);
         gap += gtot[b];
       }
       if (cur1 >= 0) {
@@ -960,14 +992,15 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       if (c + 1 < nch) {
         const int m = __ffs(~c) - 1;
         // the lower levels do not depend on this chunk: sum them before H arrives
-        float hv[16];
+        float2 hv[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) hv[e] = 0.f;
+        for (int e = 0; e < 8; ++e) hv[e] = make_float2(0.f, 0.f);
         float acc = gend;
 #pragma unroll
         for (int b = 0; b < kLevels; ++b) {
           if (b < m) {
             const float f = __expf(acc);
+            const float2 f2 = make_float2(f, f);
             const uint8_t* sl = slots + b * 8192;
 #pragma unroll
             for (int qd = 0; qd < 2; ++qd) {
@@ -978,11 +1011,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
               const uint32_t bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 ah = *reinterpret_cast<const __nv_bfloat162*>(&av[e]);
-                const __nv_bfloat162 bl = *reinterpret_cast<const __nv_bfloat162*>(&bv[e]);
-                hv[8 * qd + 2 * e] = fmaf(f, __low2float(ah) + __low2float(bl), hv[8 * qd + 2 * e]);
-                hv[8 * qd + 2 * e + 1] =
-                    fmaf(f, __high2float(ah) + __high2float(bl), hv[8 * qd + 2 * e + 1]);
+                const float2 ah = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+                const float2 bl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+                hv[4 * qd + e] = __ffma2_rn(f2, __fadd2_rn(ah, bl), hv[4 * qd + e]);
               }
             }
             acc += gtot[b];
@@ -992,12 +1023,18 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         tc_fence_after();
         {
           // H^T = V^T K_hi (columns 0..63) + V^T K_lo (64..127); this thread's 16 d_k columns
-          float t16[16], u16[16];
-          tmem_ld16(tmem + lane_off + kPColH + dk0, t16);
-          tmem_ld16(tmem + lane_off + kPColH + 64 + dk0, u16);
-          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) hv[e] += t16[e] + u16[e];
+          for (int qd = 0; qd < 2; ++qd) {
+            float t8[8], u8[8];
+            tmem_ld8(tmem + lane_off + kPColH + dk0 + 8 * qd, t8);
+            tmem_ld8(tmem + lane_off + kPColH + 64 + dk0 + 8 * qd, u8);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              hv[4 * qd + e] = __fadd2_rn(hv[4 * qd + e],
+                                          __fadd2_rn(make_float2(t8[2 * e], t8[2 * e + 1]),
+                                                     make_float2(u8[2 * e], u8[2 * e + 1])));
+          }
         }
         tc_fence_before();
         mbar_arrive(&bars[B_HEMPTY]);
@@ -1006,8 +1043,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         for (int qd = 0; qd < 2; ++qd) {
           uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            split_pack(hv[8 * qd + 2 * e], hv[8 * qd + 2 * e + 1], hi[e], lo[e]);
+          for (int e = 0; e < 4; ++e) split_pack(hv[4 * qd + e].x, hv[4 * qd + e].y, hi[e], lo[e]);
           const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
           *reinterpret_cast<uint4*>(dsl + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(dsl + kPLoOff + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -1018,17 +1054,6 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           if (b == m) gtot[b] = acc;
         mbar_arrive(&bars[(c & 1) ? B_LV1 : B_LV]);
       }
-      W(B_OFULL, c & 1);
-      tc_fence_after();
-      {
-        float r0[32];
-        tmem_ld32(tmem + lane_off + kPColO + 32 * half, r0);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] += r0[e];
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[B_OEMPTY]);
       if (n == kC) {
         // Whole chunk: stage the 128 x 64 fp32 tile in the Q (columns 0..31) and K (32..63)
         // tiles of this stage -- every reader of them is done by now -- in the 128-byte
@@ -1038,25 +1063,18 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 #pragma unroll
         for (int qd = 0; qd < 8; ++qd)
           *reinterpret_cast<float4*>(stg + row * 128 + ((qd ^ (row & 7)) << 4)) =
-              make_float4(o[4 * qd], o[4 * qd + 1], o[4 * qd + 2], o[4 * qd + 3]);
+              make_float4(o2[2 * qd].x, o2[2 * qd].y, o2[2 * qd + 1].x, o2[2 * qd + 1].y);
         fence_proxy_async_smem();
-        named_sync(2, kPNB);
-        if (warp == kPB0 && lane == 0) {
-          const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
-          tma_store_3d(&tmo, stage(s), 0, h, tok0);
-          tma_store_3d(&tmo, stage(s) + kTile, 32, h, tok0);
-          bulk_commit();
-          bulk_wait_read();
-          mbar_arrive(&bars[B_EMPTY + s]);  // the stage may be refilled
-        }
+        mbar_arrive(&bars[B_OSTAGED + s]);  // the producer stores the tile
       } else {
         if (row < n) {
           float* dst = out + ((sp.start + (long long)c * kC + row) * H + h) * kD + 32 * half;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+          for (int e = 0; e < 16; e += 2)
+            *reinterpret_cast<float4*>(dst + 2 * e) =
+                make_float4(o2[e].x, o2[e].y, o2[e + 1].x, o2[e + 1].y);
         }
-        if (warp == kPB0 && lane == 0) mbar_arrive(&bars[B_EMPTY + s]);
+        mbar_arrive(&bars[B_OSTAGED + s]);  // nothing staged; keeps the phases in step
       }
       mbar_arrive(&bars[B_GEMPTY + c % kPG]);
     }
@@ -1110,7 +1128,6 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     }
   }
 
-  if (warp == kPB0 && lane == 0) bulk_wait_all();  // output tiles written
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
