@@ -765,8 +765,23 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     // K scaling warp.
     float g_row = 0.f, g0 = 0.f, gend = 0.f;
     bool factored = true;
+    // L2 prefetch of chunk cc's lam and log a.  For one head the rows of a chunk are short
+    // pieces far apart; across the H heads they form one contiguous block per chunk, so each
+    // head's CTA pulls its 1/H share of the block, and the per-row loads then hit L2.  Whole
+    // chunks only (the block lies inside the tensors), and only where the 16-byte rule of
+    // bulk copies holds; it is a hint and changes no result.
+    auto l2_prefetch = [&](int cc) {
+      if (cc >= nch || !is_full(cc)) return;
+      const long long tok0 = sp.start + (long long)cc * kC;
+      const float* lb = lam + (tok0 * H + (long long)h * kC) * L;    // share h of the block
+      const float* ab = log_a + tok0 * H + (long long)h * kC;
+      if (((reinterpret_cast<uintptr_t>(lb) | (uint32_t)(kC * L * 4)) & 15u) == 0)
+        bulk_prefetch_l2(lb, kC * L * 4);
+      if ((reinterpret_cast<uintptr_t>(ab) & 15u) == 0) bulk_prefetch_l2(ab, kC * 4);
+    };
     auto decay_scan = [&](int c) {
       const int gb = c % kPG, gk = c / kPG;  // g buffer and its use index
+      if (wa == 0 && lane == 0) l2_prefetch(c + 2);
       const int n = min(kC, sp.len - c * kC);
       float pfc[kNP];
 #pragma unroll
@@ -808,6 +823,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         lamB[(gb * kC + row) * kLevels + part + 2 * i - (kLogC + 1)] = pfc[i] * eg;
       mbar_arrive(&bars[B_GREADY + gb]);
     };
+    if (wa == 0 && lane == 0) l2_prefetch(1);
     prefetch(0);
     decay_scan(0);
     for (int c = 0; c < nch; ++c) {
