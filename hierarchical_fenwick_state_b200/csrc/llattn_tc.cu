@@ -955,7 +955,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     for (int b = 0; b < kLevels; ++b) gtot[b] = 0.f;
     uint32_t u = 0;
     for (int c = 0; c < nch; ++c) {
-      const int s = c & 1, kk = c >> 1;
+      const int s = c & 1;
       const int n = min(kC, sp.len - c * kC);
       W(B_GREADY + c % kPG, (c / kPG) & 1);
       const float gend = gs[(c % kPG) * kC + n - 1];
