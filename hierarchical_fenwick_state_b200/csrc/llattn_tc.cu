@@ -27,6 +27,7 @@
 // the result within fp32-accumulation error of the exact sum; out is fp32.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -90,6 +91,22 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t& hi, uint3
   const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u, ub = __float_as_uint(b) & 0xFFFF0000u;
   hi = __byte_perm(ua, ub, 0x7632);  // high halves of a (low) and b (high)
   lo = pack_bf16(a - __uint_as_float(ua), b - __uint_as_float(ub));
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);  // a -> low 16 bits
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 8 bf16 values (a uint4) -> 8 fp16 values
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 x) {
+  uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+    w[e] = pack_f16(f.x, f.y);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __device__ __forceinline__ float bf16_at(const uint8_t* p) {
@@ -514,8 +531,7 @@ constexpr int kPB0 = 10;                      // first warp of group B
 constexpr int kPNB = 8 * 32;                  // group B threads
 constexpr int kPI2 = 18;                      // warp of the inter-chunk MMA issuer
 
-constexpr uint32_t kPOffKlo = 2 * kStage;
-constexpr uint32_t kPOffSlots = kPOffKlo + kTile;   // level hi parts, then level lo parts
+constexpr uint32_t kPOffSlots = 2 * kStage;         // level hi parts, then level lo parts
 constexpr uint32_t kPLoOff = kLevels * 8192;        // lo part of level b at + kPLoOff + b * 8 KB
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
 constexpr uint32_t kPOffLam = kPOffSlots + kLevels * kSlot;
@@ -531,13 +547,16 @@ constexpr int kPNumBars = 27;
 constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
 constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
 
-constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (hi/lo)
+constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (fp16)
 constexpr uint32_t kPColO = 128;   // P V accumulator
-constexpr uint32_t kPColH = 192;   // V^T [K_hi | K_lo] (128 cols), rows duplicated in lanes 64..127
-constexpr uint32_t kPColR = 320;   // readout accumulator: up to three adjacent levels
-constexpr int kPSpan = 3;          // levels one readout chain covers (N = 64 per level)
+constexpr uint32_t kPColH = 192;   // V^T K~, rows duplicated in lanes 64..127
+constexpr uint32_t kPColR = 256;   // readout accumulator: up to four adjacent levels
+constexpr int kPSpan = 4;          // levels one readout chain covers (N = 64 per level)
 
-constexpr uint32_t kIdescHT = idesc_bf16(128, 128, 1, 1);  // V^T (M contiguous) x [K_hi | K_lo]
+// P V and the chunk state run in fp16: V is converted in place when its tile lands, P and
+// the decay-scaled K are rounded once to fp16 (10-bit mantissa; no hi/lo split needed)
+constexpr uint32_t kIdescHT = idesc_f16(128, 64, 1, 1);   // V^T (M contiguous) x K~ (N contiguous)
+constexpr uint32_t kIdescPVh = idesc_f16(128, 64, 0, 1);  // P (TMEM) x V (N contiguous)
 
 enum : int {
   B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 5, B_SPEMPTY = 6, B_KS = 7, B_HFULL = 8,
@@ -616,7 +635,6 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   const int nch = (sp.len + kC - 1) / kC;
 
   auto stage = [sm](int i) { return sm + i * kStage; };
-  uint8_t* klo = sm + kPOffKlo;
   uint8_t* slots = sm + kPOffSlots;
   float* lamA = reinterpret_cast<float*>(sm + kPOffLam);
   float* gs = reinterpret_cast<float*>(sm + kPOffG);
@@ -716,14 +734,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         const int s = c & 1;
         if (!W(B_PFULL, c & 1) || !W(B_OEMPTY, (c & 1) ^ 1)) break;
         tc_fence_after();
-        // K-step x covers keys 16x..16x+15: hi in columns 16x..16x+7, lo in 16x+8..16x+15
+        // K-step x covers keys 16x..16x+15, their fp16 P in columns 16x..16x+7
         const uint64_t vd = mndesc(smem_u32(stage(s)) + 2 * kTile);
 #pragma unroll
         for (int x = 0; x < kC / 16; ++x)
-          mma_ts(tmem + kPColO, tmem + kPColSP + 16 * x, vd + 128 * x, kIdescPV, x > 0);
-#pragma unroll
-        for (int x = 0; x < kC / 16; ++x)
-          mma_ts(tmem + kPColO, tmem + kPColSP + 16 * x + 8, vd + 128 * x, kIdescPV, 1);
+          mma_ts(tmem + kPColO, tmem + kPColSP + 16 * x, vd + 128 * x, kIdescPVh, x > 0);
         mma_commit(&bars[B_OFULL]);
         mma_commit(&bars[B_SPEMPTY]);
         mma_commit(&bars[B_EMPTY + s]);   // this issuer's reads of stage s are done
@@ -841,8 +856,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           for (int j = 0; j < 4; ++j) {
             const int col = part * 32 + j * 8;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (row < n)
+            if (row < n) {
               val = *reinterpret_cast<const uint4*>(src + ((tok0 + row) * H + h) * kD + col);
+              if (tsr == 2) val = bf16x8_to_f16x8(val);   // V in fp16
+            }
             *reinterpret_cast<uint4*>(stage(s) + tsr * kTile + sw128_off(row, col)) = val;
           }
         }
@@ -851,6 +868,14 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         if (wa == 0 && lane == 0) mbar_arrive(&bars[B_FULL + s]);
       }
       W(B_FULL + s, kk & 1);
+      if (is_full(c)) {
+        // V to fp16 in place (the element layout is the same), while S(c) runs
+        uint4* vt = reinterpret_cast<uint4*>(stage(s) + 2 * kTile);
+        const int t = wa * 32 + lane;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) vt[t + 256 * i] = bf16x8_to_f16x8(vt[t + 256 * i]);
+        fence_proxy_async_smem();
+      }
       W(B_SFULL, c & 1);
       tc_fence_after();
       named_sync(1, kPNA);  // cj and the lam table are visible to the whole group
@@ -863,10 +888,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 #pragma unroll 1
       for (int g16 = part; g16 < 8; g16 += 2) {  // keys 16*g16 .. 16*g16+15
         const int kb = g16 >> 1;                // their 32-key block
-        uint32_t hi[8], lo[8];
+        uint32_t hi[8];
         if (kb > rb) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) { hi[e] = 0u; lo[e] = 0u; }
+          for (int e = 0; e < 8; ++e) hi[e] = 0u;
         } else {
           float sv[16];
           tmem_ld16(spc + 16 * g16, sv);
@@ -889,7 +914,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             const float wblk = lr[6 + (31 - __clz(rb ^ kb))];
 #pragma unroll
             for (int e = 0; e < 16; e += 2)
-              split_pack(sv[e] * wblk * cw[e], sv[e + 1] * wblk * cw[e + 1], hi[e >> 1], lo[e >> 1]);
+              hi[e >> 1] = pack_f16(sv[e] * wblk * cw[e], sv[e + 1] * wblk * cw[e + 1]);
           } else {
             // diagonal block: level 1 + msb(lane ^ jj) (0 when equal: clz(0) = 32), j <= i
             const int j0 = 16 * (g16 & 1);
@@ -902,12 +927,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
                 const float val = sv[e + t2] * lr[32 - __clz(jj ^ lane)] * cw[e + t2];
                 p[t2] = jj <= lane ? val : 0.f;
               }
-              split_pack(p[0], p[1], hi[e >> 1], lo[e >> 1]);
+              hi[e >> 1] = pack_f16(p[0], p[1]);
             }
           }
         }
         tmem_st8(spc + 16 * g16, hi);
-        tmem_st8(spc + 16 * g16 + 8, lo);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -919,7 +943,6 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       // mask loads sub-partitions 0..3 in the ratio 1:2:3:4, so the K rows are dealt out the
       // other way round: 48, 40, 24 and 16 rows to the two warps of sub-partitions 0..3.
       if (c + 1 < nch) {
-        if (c > 0) W(B_HFULL, (c - 1) & 1);   // H of the previous chunk has read klo
         uint8_t* kt = stage(s) + kTile;
         const int r0 = sub == 0 ? 0 : (sub == 1 ? 48 : (sub == 2 ? 88 : 112));
         const int nrows = sub == 0 ? 48 : (sub == 1 ? 40 : (sub == 2 ? 24 : 16));
@@ -931,14 +954,13 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           const uint32_t off = sw128_off(kr, (unit & 7) * 8);
           const uint4 raw = *reinterpret_cast<const uint4*>(kt + off);
           const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t hi[4], lo[4];
+          uint32_t hv4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
-            split_pack(__low2float(pr) * ks, __high2float(pr) * ks, hi[e], lo[e]);
+            const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+            hv4[e] = pack_f16(pr.x * ks, pr.y * ks);
           }
-          *reinterpret_cast<uint4*>(kt + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(klo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(kt + off) = make_uint4(hv4[0], hv4[1], hv4[2], hv4[3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars[B_KS]);
@@ -1038,19 +1060,13 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         W(B_HFULL, c & 1);
         tc_fence_after();
         {
-          // H^T = V^T K_hi (columns 0..63) + V^T K_lo (64..127); this thread's 16 d_k columns
+          // H^T = V^T K~; this thread's 16 d_k columns
+          float t16[16];
+          tmem_ld16(tmem + lane_off + kPColH + dk0, t16);
+          tmem_wait_ld();
 #pragma unroll
-          for (int qd = 0; qd < 2; ++qd) {
-            float t8[8], u8[8];
-            tmem_ld8(tmem + lane_off + kPColH + dk0 + 8 * qd, t8);
-            tmem_ld8(tmem + lane_off + kPColH + 64 + dk0 + 8 * qd, u8);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              hv[4 * qd + e] = __fadd2_rn(hv[4 * qd + e],
-                                          __fadd2_rn(make_float2(t8[2 * e], t8[2 * e + 1]),
-                                                     make_float2(u8[2 * e], u8[2 * e + 1])));
-          }
+          for (int e = 0; e < 8; ++e)
+            hv[e] = __fadd2_rn(hv[e], make_float2(t16[2 * e], t16[2 * e + 1]));
         }
         tc_fence_before();
         mbar_arrive(&bars[B_HEMPTY]);
@@ -1130,9 +1146,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         if (c + 1 < nch) {
           if (!W(B_KS, c & 1) || !W(B_HEMPTY, (c & 1) ^ 1)) break;
           tc_fence_after();
-          // B = [K_hi | K_lo]: two 64-wide N groups, the second at the klo tile (LBO)
+          // A = V^T (fp16, rows duplicated), B = K~ (fp16, in the K tile)
           const uint64_t vd = mndesc_dup(va);
-          const uint64_t kd = sdesc_sw128(ka, smem_u32(klo) - ka, 1024);
+          const uint64_t kd = mndesc(ka);
 #pragma unroll
           for (int x = 0; x < kC / 16; ++x) mma_ss(tmem + kPColH, vd + 128 * x, kd + 128 * x, kIdescHT, x > 0);
           mma_commit(&bars[B_HFULL]);

@@ -277,6 +277,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | (uint32_t(M >> 4) << 24);     // M / 16
 }
 
+// The same for fp16 A and B operands (kind::f16, f32 accumulate).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                       // D format: f32 (A, B format 0: f16)
+         | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) |
+         (uint32_t(M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand.
 // K-major: rows of 128 B (64 bf16 along K), 8-row atoms of 1024 B, sbo = 1024;
 // MN-major: rows of 128 B along M/N, 8 rows of K per atom, sbo = 1024 between
