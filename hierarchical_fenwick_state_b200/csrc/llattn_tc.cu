@@ -531,10 +531,10 @@ constexpr int kPB0 = 10;                      // first warp of group B
 constexpr int kPNB = 8 * 32;                  // group B threads
 constexpr int kPI2 = 18;                      // warp of the inter-chunk MMA issuer
 
-constexpr uint32_t kPOffSlots = 2 * kStage;         // level hi parts, then level lo parts
-constexpr uint32_t kPLoOff = kLevels * 8192;        // lo part of level b at + kPLoOff + b * 8 KB
+constexpr uint32_t kPOffSlots = 2 * kStage;         // level states, fp16 [d_v rows][d_k], 8 KB each
+constexpr uint32_t kPOffQh = kPOffSlots + kLevels * 8192;  // fp16 copy of Q for the readouts
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
-constexpr uint32_t kPOffLam = kPOffSlots + kLevels * kSlot;
+constexpr uint32_t kPOffLam = kPOffQh + kTile;
 constexpr int kPG = 3;                                         // g buffers
 constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[3][128]
 constexpr uint32_t kPOffCj = kPOffG + kPG * kC * 4;
@@ -636,6 +636,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 
   auto stage = [sm](int i) { return sm + i * kStage; };
   uint8_t* slots = sm + kPOffSlots;
+  uint8_t* qh = sm + kPOffQh;
   float* lamA = reinterpret_cast<float*>(sm + kPOffLam);
   float* gs = reinterpret_cast<float*>(sm + kPOffG);
   float* cj = reinterpret_cast<float*>(sm + kPOffCj);
@@ -1044,14 +1045,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             for (int qd = 0; qd < 2; ++qd) {
               const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
               const uint4 a4 = *reinterpret_cast<const uint4*>(sl + off);
-              const uint4 b4 = *reinterpret_cast<const uint4*>(sl + kPLoOff + off);
               const uint32_t av[4] = {a4.x, a4.y, a4.z, a4.w};
-              const uint32_t bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const float2 ah = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
-                const float2 bl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
-                hv[4 * qd + e] = __ffma2_rn(f2, __fadd2_rn(ah, bl), hv[4 * qd + e]);
+                const float2 ah = __half22float2(*reinterpret_cast<const __half2*>(&av[e]));
+                hv[4 * qd + e] = __ffma2_rn(f2, ah, hv[4 * qd + e]);
               }
             }
             acc += gtot[b];
@@ -1073,12 +1071,21 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         uint8_t* dsl = slots + m * 8192;
 #pragma unroll
         for (int qd = 0; qd < 2; ++qd) {
-          uint32_t hi[4], lo[4];
+          uint32_t hh[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) split_pack(hv[4 * qd + e].x, hv[4 * qd + e].y, hi[e], lo[e]);
+          for (int e = 0; e < 4; ++e) hh[e] = pack_f16(hv[4 * qd + e].x, hv[4 * qd + e].y);
           const uint32_t off = sw128_off(j_dv, dk0 + 8 * qd);
-          *reinterpret_cast<uint4*>(dsl + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(dsl + kPLoOff + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(dsl + off) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+        }
+        // fp16 copy of Q(c + 1) for its readouts: every readout of chunk c has been drained,
+        // and the level-ready signal below also releases this copy to the MMA issuer
+        W(B_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+        {
+          const uint4* qsrc = reinterpret_cast<const uint4*>(stage((c + 1) & 1));
+          uint4* qdst = reinterpret_cast<uint4*>(qh);
+          const int t = (warp - kPB0) * 32 + lane;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) qdst[t + 256 * i] = bf16x8_to_f16x8(qsrc[t + 256 * i]);
         }
         fence_proxy_async_smem();
 #pragma unroll
@@ -1131,14 +1138,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             break;
           }
           tc_fence_after();
-          const uint64_t qd = kdesc(qa);
+          const uint64_t qd = kdesc(smem_u32(qh));   // fp16 copy of Q(c)
           const uint64_t sd = kdesc(smem_u32(slots + cb0 * 8192));
-          const uint64_t sdl = kdesc(smem_u32(slots + kPLoOff + cb0 * 8192));
-          const uint32_t idr = idesc_bf16(128, 64 * (cb1 - cb0 + 1), 0, 0);
+          const uint32_t idr = idesc_f16(128, 64 * (cb1 - cb0 + 1), 0, 0);
 #pragma unroll
           for (int x = 0; x < kD / 16; ++x) mma_ss(tmem + kPColR, qd + 2 * x, sd + 2 * x, idr, x > 0);
-#pragma unroll
-          for (int x = 0; x < kD / 16; ++x) mma_ss(tmem + kPColR, qd + 2 * x, sdl + 2 * x, idr, 1);
           mma_commit(&bars[B_RFULL]);
           ++u;
         }
