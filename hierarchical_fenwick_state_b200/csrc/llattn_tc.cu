@@ -512,7 +512,7 @@ tc_fwd_serial(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
 
 // ==========================================================================================
 // Pipelined variant: warp-specialised roles linked by mbarriers.
-//   warp 0        TMA producer (Q, K, V tiles of chunk c into stage c % 2)
+//   warp 0        TMA producer (Q, K, V tiles of chunk c into stage c % 3; output tiles out)
 //   warp 1        MMA issuer for the intra-chunk part (S, P V)
 //   warp 18       MMA issuer for the inter-chunk part (H^T, level readouts)
 //   warps 2..9    group A      (decay scan, K scaling for the chunk state, causal mask -> P)
@@ -531,7 +531,8 @@ constexpr int kPB0 = 10;                      // first warp of group B
 constexpr int kPNB = 8 * 32;                  // group B threads
 constexpr int kPI2 = 18;                      // warp of the inter-chunk MMA issuer
 
-constexpr uint32_t kPOffSlots = 2 * kStage;         // level states, fp16 [d_v rows][d_k], 8 KB each
+constexpr int kPStages = 3;                          // Q/K/V ring: chunk c in stage c % 3
+constexpr uint32_t kPOffSlots = kPStages * kStage;   // level states, fp16 [d_v rows][d_k], 8 KB each
 constexpr uint32_t kPOffQh = kPOffSlots + kLevels * 8192;  // fp16 copy of Q for the readouts
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
 constexpr uint32_t kPOffLam = kPOffQh + kTile;
@@ -543,9 +544,10 @@ constexpr uint32_t kPOffCj = kPOffG + kPG * kC * 4;
 constexpr uint32_t kPOffLamB = kPOffCj + kC * 4;
 constexpr uint32_t kPOffScan = kPOffLamB + kPG * kC * kLevels * 4;
 constexpr uint32_t kPOffBar = kPOffScan + 64;
-constexpr int kPNumBars = 27;
+constexpr int kPNumBars = 30;
 constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
 constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
+static_assert(kPSmemBytes <= 227 * 1024, "shared memory of the pipelined kernel exceeds 227 KB");
 
 constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (fp16)
 constexpr uint32_t kPColO = 128;   // P V accumulator
@@ -559,10 +561,10 @@ constexpr uint32_t kIdescHT = idesc_f16(128, 64, 1, 1);   // V^T (M contiguous) 
 constexpr uint32_t kIdescPVh = idesc_f16(128, 64, 0, 1);  // P (TMEM) x V (N contiguous)
 
 enum : int {
-  B_FULL = 0, B_EMPTY = 2, B_SFULL = 4, B_PFULL = 5, B_SPEMPTY = 6, B_KS = 7, B_HFULL = 8,
-  B_HEMPTY = 9, B_LV = 10, B_LV1 = 11, B_OFULL = 12, B_OEMPTY = 13, B_RFULL = 14,
-  B_REMPTY = 15, B_GREADY = 16, B_GEMPTY = 19, B_DRAIN = 22, B_DRAIN2 = 23, B_OSTAGED = 24,
-  B_FREE = 26
+  B_FULL = 0, B_EMPTY = 3, B_SFULL = 6, B_PFULL = 7, B_SPEMPTY = 8, B_KS = 9, B_HFULL = 10,
+  B_HEMPTY = 11, B_LV = 12, B_LV1 = 13, B_OFULL = 14, B_OEMPTY = 15, B_RFULL = 16,
+  B_REMPTY = 17, B_GREADY = 18, B_GEMPTY = 21, B_DRAIN = 24, B_DRAIN2 = 25, B_OSTAGED = 26,
+  B_FREE = 29
 };
 
 // Wait on an mbarrier phase; returns false at once if the CTA has aborted, and aborts
@@ -653,10 +655,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   if (tid == 32) {
     for (int i = 0; i < kPNumBars; ++i) {
       uint32_t cnt = 1;  // TMA / tcgen05.commit arrivals
-      if (i == B_EMPTY || i == B_EMPTY + 1) cnt = 2;  // both MMA issuers
+      if (i >= B_EMPTY && i < B_EMPTY + kPStages) cnt = 2;  // both MMA issuers
       if (i == B_PFULL || i == B_KS || (i >= B_GREADY && i < B_GREADY + kPG)) cnt = kPNA;
       if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY || i == B_REMPTY ||
-          (i >= B_GEMPTY && i < B_GEMPTY + kPG) || i == B_OSTAGED || i == B_OSTAGED + 1)
+          (i >= B_GEMPTY && i < B_GEMPTY + kPG) || (i >= B_OSTAGED && i < B_OSTAGED + kPStages))
         cnt = kPNB;
       mbar_init(&bars[i], cnt);
     }
@@ -675,28 +677,28 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    // Loads Q, K, V of chunk c into stage c % 2 once that stage is free: both MMA issuers are
-    // done with chunk c - 2, whose output tile group B staged there, and this thread has
+    // Loads Q, K, V of chunk c into stage c % 3 once that stage is free: both MMA issuers are
+    // done with chunk c - 3, whose output tile group B staged there, and this thread has
     // stored that tile (TMA store, waited until its shared-memory reads are done).  Doing the
     // store here keeps its wait out of group B's chunk loop.  A ragged last chunk is loaded
     // by group A with plain loads; B_FREE tells it the stage is free.
     if (lane == 0) {
-      int last0 = -1, last1 = -1;
+      int last0 = -1, last1 = -1, last2 = -1;
       bool ok = true;
       auto store_out = [&](int cc) {
-        if (!W(B_OSTAGED + (cc & 1), (cc >> 1) & 1)) return false;
+        if (!W(B_OSTAGED + cc % kPStages, (cc / kPStages) & 1)) return false;
         if (is_full(cc)) {
           const int tok0 = static_cast<int>(sp.start + (long long)cc * kC);
-          tma_store_3d(&tmo, stage(cc & 1), 0, h, tok0);
-          tma_store_3d(&tmo, stage(cc & 1) + kTile, 32, h, tok0);
+          tma_store_3d(&tmo, stage(cc % kPStages), 0, h, tok0);
+          tma_store_3d(&tmo, stage(cc % kPStages) + kTile, 32, h, tok0);
           bulk_commit();
           bulk_wait_read();
         }
         return true;
       };
       for (int c = 0; c < nch; ++c) {
-        const int s = c & 1, kk = c >> 1;
-        if (c >= 2 && (!W(B_EMPTY + s, (kk & 1) ^ 1) || !store_out(c - 2))) {
+        const int s = c % kPStages, kk = c / kPStages;
+        if (c >= kPStages && (!W(B_EMPTY + s, (kk & 1) ^ 1) || !store_out(c - kPStages))) {
           ok = false;
           break;
         }
@@ -706,17 +708,18 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           tma_load_3d(stage(s), &tmq, &bars[B_FULL + s], 0, h, tok0);
           tma_load_3d(stage(s) + kTile, &tmk, &bars[B_FULL + s], 0, h, tok0);
           tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[B_FULL + s], 0, h, tok0);
-          if (s == 0) last0 = c; else last1 = c;
+          if (s == 0) last0 = c; else if (s == 1) last1 = c; else last2 = c;
         } else {
           mbar_arrive(&bars[B_FREE]);
         }
       }
-      for (int cc = nch > 2 ? nch - 2 : 0; ok && cc < nch; ++cc) ok = store_out(cc);
+      for (int cc = nch > kPStages ? nch - kPStages : 0; ok && cc < nch; ++cc) ok = store_out(cc);
       bulk_wait_all();  // output tiles written
       if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) {
         // an aborted CTA still lets its own copies land before it exits
-        if (last0 >= 0) mbar_wait(&bars[B_FULL + 0], (last0 >> 1) & 1, 200000000ull);
-        if (last1 >= 0) mbar_wait(&bars[B_FULL + 1], (last1 >> 1) & 1, 200000000ull);
+        if (last0 >= 0) mbar_wait(&bars[B_FULL + 0], (last0 / kPStages) & 1, 200000000ull);
+        if (last1 >= 0) mbar_wait(&bars[B_FULL + 1], (last1 / kPStages) & 1, 200000000ull);
+        if (last2 >= 0) mbar_wait(&bars[B_FULL + 2], (last2 / kPStages) & 1, 200000000ull);
       }
     }
   } else if (warp == 1) {
@@ -732,7 +735,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         mma_commit(&bars[B_SFULL]);
       }
       for (int c = 0; ok && c < nch; ++c) {
-        const int s = c & 1;
+        const int s = c % kPStages;
         if (!W(B_PFULL, c & 1) || !W(B_OEMPTY, (c & 1) ^ 1)) break;
         tc_fence_after();
         // K-step x covers keys 16x..16x+15, their fp16 P in columns 16x..16x+7
@@ -744,8 +747,8 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         mma_commit(&bars[B_SPEMPTY]);
         mma_commit(&bars[B_EMPTY + s]);   // this issuer's reads of stage s are done
         if (c + 1 < nch) {
-          const int s1 = (c + 1) & 1;
-          if (!W(B_FULL + s1, ((c + 1) >> 1) & 1) || !W(B_SPEMPTY, c & 1)) break;
+          const int s1 = (c + 1) % kPStages;
+          if (!W(B_FULL + s1, ((c + 1) / kPStages) & 1) || !W(B_SPEMPTY, c & 1)) break;
           tc_fence_after();
           const uint64_t qd = kdesc(smem_u32(stage(s1))), kd = kdesc(smem_u32(stage(s1)) + kTile);
 #pragma unroll
@@ -843,11 +846,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     prefetch(0);
     decay_scan(0);
     for (int c = 0; c < nch; ++c) {
-      const int s = c & 1, kk = c >> 1;
+      const int s = c % kPStages, kk = c / kPStages;
       const int n = min(kC, sp.len - c * kC);
       if (!is_full(c)) {
         // ragged last chunk: plain loads into the stage, rows past the end zero-filled, once
-        // the producer has stored the output tile of chunk c - 2 from it
+        // the producer has stored the output tile of chunk c - 3 from it
         W(B_FREE, 0);
         const long long tok0 = sp.start + (long long)c * kC;
 #pragma unroll
@@ -944,6 +947,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       // mask loads sub-partitions 0..3 in the ratio 1:2:3:4, so the K rows are dealt out the
       // other way round: 48, 40, 24 and 16 rows to the two warps of sub-partitions 0..3.
       if (c + 1 < nch) {
+        // H^T(c - 1) must be done before K scaling (c) is signalled: the MMA issuer waits for
+        // the K-scaled barrier once per chunk, so this group may run at most one phase ahead
+        if (c > 0) W(B_HFULL, (c - 1) & 1);
         uint8_t* kt = stage(s) + kTile;
         const int r0 = sub == 0 ? 0 : (sub == 1 ? 48 : (sub == 2 ? 88 : 112));
         const int nrows = sub == 0 ? 48 : (sub == 1 ? 40 : (sub == 2 ? 24 : 16));
@@ -978,7 +984,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     for (int b = 0; b < kLevels; ++b) gtot[b] = 0.f;
     uint32_t u = 0;
     for (int c = 0; c < nch; ++c) {
-      const int s = c & 1;
+      const int s = c % kPStages;
       const int n = min(kC, sp.len - c * kC);
       W(B_GREADY + c % kPG, (c / kPG) & 1);
       const float gend = gs[(c % kPG) * kC + n - 1];
@@ -1079,9 +1085,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         }
         // fp16 copy of Q(c + 1) for its readouts: every readout of chunk c has been drained,
         // and the level-ready signal below also releases this copy to the MMA issuer
-        W(B_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+        W(B_FULL + (c + 1) % kPStages, ((c + 1) / kPStages) & 1);
         {
-          const uint4* qsrc = reinterpret_cast<const uint4*>(stage((c + 1) & 1));
+          const uint4* qsrc = reinterpret_cast<const uint4*>(stage((c + 1) % kPStages));
           uint4* qdst = reinterpret_cast<uint4*>(qh);
           const int t = (warp - kPB0) * 32 + lane;
 #pragma unroll
@@ -1126,8 +1132,8 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     if (lane == 0) {
       uint32_t u = 0;  // readout chains issued so far
       for (int c = 0; c < nch; ++c) {
-        const int s = c & 1;
-        if (!W(B_FULL + s, (c >> 1) & 1)) break;
+        const int s = c % kPStages;
+        if (!W(B_FULL + s, (c / kPStages) & 1)) break;
         const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile, va = qa + 2 * kTile;
         bool ok = true;
         int cb0 = 0, cb1 = 0;
