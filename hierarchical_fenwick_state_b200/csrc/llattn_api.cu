@@ -62,7 +62,10 @@ llattn_status resolve(int in_dtype, int* path, int* chunk, int T, int dk, int dv
     if (*chunk < 8 || *chunk > 64) return LLATTN_ERR_ARG;
   } else {
     if (in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
-    if (!llattn::tc_supports(in_dtype, dk, dv, *chunk, T)) return LLATTN_ERR_UNSUPPORTED;
+    const bool ok = *path == LLATTN_PATH_TCGEN05_SERIAL
+                        ? llattn::tc_serial_supports(in_dtype, dk, dv, *chunk, T)
+                        : llattn::tc_supports(in_dtype, dk, dv, *chunk, T);
+    if (!ok) return LLATTN_ERR_UNSUPPORTED;
   }
   return LLATTN_OK;
 }

@@ -36,6 +36,7 @@ size_t tc_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk);
 cudaError_t simt_forward(const Problem& p, int chunk, void* ws, cudaStream_t st);
 cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, bool serial);
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T);
+bool tc_serial_supports(int in_dtype, int dk, int dv, int chunk, int T);
 
 // Device address of the fixed scratch array behind llattn_fwd_noalloc on the
 // current device (looked up on the first call per device, then cached).

@@ -541,23 +541,31 @@ constexpr int kPB0 = 10;                      // first warp of group B
 constexpr int kPNB = 8 * 32;                  // group B threads
 constexpr int kPI2 = 18;                      // warp of the inter-chunk MMA issuer
 
-constexpr int kPStages = 3;                          // Q/K/V ring: chunk c in stage c % 3
-constexpr uint32_t kPOffSlots = kPStages * kStage;   // level states, fp16 [d_v rows][d_k], 8 KB each
-constexpr uint32_t kPOffQh = kPOffSlots + kLevels * 8192;  // fp16 copy of Q for the readouts
+constexpr int kPG = 3;                        // g buffers
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
-constexpr uint32_t kPOffLam = kPOffQh + kTile;
-constexpr int kPG = 3;                                         // g buffers
-constexpr uint32_t kPOffG = kPOffLam + kC * kPLamStride * 4;   // g[3][128]
-constexpr uint32_t kPOffCj = kPOffG + kPG * kC * 4;
-// lam of the inter-chunk levels 1+log2 C+b (b < kLevels) times exp(g_i), per row: group A
-// writes it with the decay scan, group B reads it for the readout weights (g buffers' ring)
-constexpr uint32_t kPOffLamB = kPOffCj + kC * 4;
-constexpr uint32_t kPOffScan = kPOffLamB + kPG * kC * kLevels * 4;
-constexpr uint32_t kPOffBar = kPOffScan + 64;
 constexpr int kPNumBars = 30;
-constexpr uint32_t kPOffMisc = kPOffBar + kPNumBars * 8;
-constexpr uint32_t kPSmemBytes = kPOffMisc + 64 + 1024;
-static_assert(kPSmemBytes <= 227 * 1024, "shared memory of the pipelined kernel exceeds 227 KB");
+
+// Shared-memory map of the pipelined kernel for NLEV chunk-level Fenwick states kept on chip
+// (T <= 128 * 2^NLEV) and an NST-stage Q/K/V ring (chunk c in stage c % NST).
+template <int NLEV, int NST>
+struct PipeLayout {
+  static constexpr int kLev = NLEV, kSt = NST;
+  static constexpr uint32_t kOffSlots = NST * kStage;         // level states, fp16 [d_v][d_k], 8 KB
+  static constexpr uint32_t kOffQh = kOffSlots + NLEV * 8192;  // fp16 copy of Q for the readouts
+  static constexpr uint32_t kOffLam = kOffQh + kTile;
+  static constexpr uint32_t kOffG = kOffLam + kC * kPLamStride * 4;   // g[3][128]
+  static constexpr uint32_t kOffCj = kOffG + kPG * kC * 4;
+  // lam of the inter-chunk levels 1+log2 C+b (b < NLEV) times exp(g_i), per row: group A
+  // writes it with the decay scan, group B reads it for the readout weights (g buffers' ring)
+  static constexpr uint32_t kOffLamB = kOffCj + kC * 4;
+  static constexpr uint32_t kOffScan = kOffLamB + kPG * kC * NLEV * 4;
+  static constexpr uint32_t kOffBar = kOffScan + 64;
+  static constexpr uint32_t kOffMisc = kOffBar + kPNumBars * 8;
+  static constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory of the pipelined kernel exceeds 227 KB");
+};
+using PipeShort = PipeLayout<6, 3>;   // T <= 8192
+using PipeLong = PipeLayout<7, 2>;    // T <= 16384
 
 constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (fp16)
 constexpr uint32_t kPColO = 128;   // P V accumulator
@@ -609,13 +617,14 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 // bit b0 of c and covers the set bits below b0 + kPSpan; its N = 64 * (b1 - b0 + 1)
 // columns read the consecutive hi (then lo) level arrays in one MMA per K step.  A level
 // inside the range whose bit is clear is computed and ignored.
+template <int NLEV>
 __device__ __forceinline__ bool next_chain(int c, int from, int& b0, int& b1) {
   int b = from;
-  while (b < kLevels && !((c >> b) & 1)) ++b;
-  if (b >= kLevels) return false;
+  while (b < NLEV && !((c >> b) & 1)) ++b;
+  if (b >= NLEV) return false;
   b0 = b;
   b1 = b;
-  for (int x = b + 1; x < kLevels && x < b + kPSpan; ++x)
+  for (int x = b + 1; x < NLEV && x < b + kPSpan; ++x)
     if ((c >> x) & 1) b1 = x;
   return true;
 }
@@ -624,6 +633,7 @@ __device__ __forceinline__ bool next_chain(int c, int from, int& b0, int& b1) {
 // an M = 128 MMA over a 64-wide operand yields the 64-row result twice.
 __device__ __forceinline__ uint64_t mndesc_dup(uint32_t saddr) { return sdesc_sw128(saddr, 0, 1024); }
 
+template <int NLEV, int NST>
 __global__ void __maxnreg__(96)
 tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
             const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
@@ -632,6 +642,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             const float* __restrict__ log_a, const float* __restrict__ lam,
             float* __restrict__ out, int H, int T, int L, const int* __restrict__ cu,
             unsigned int* status) {
+  using LY = PipeLayout<NLEV, NST>;
+  constexpr int kLevels = NLEV;   // chunk-level states on chip in this instantiation
+  constexpr int kPStages = NST;   // Q/K/V ring stages
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, by pointer arithmetic on the shared array so that the compiler
   // keeps shared-memory (not generic) loads and stores for everything derived from it
@@ -647,15 +660,15 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   const int nch = (sp.len + kC - 1) / kC;
 
   auto stage = [sm](int i) { return sm + i * kStage; };
-  uint8_t* slots = sm + kPOffSlots;
-  uint8_t* qh = sm + kPOffQh;
-  float* lamA = reinterpret_cast<float*>(sm + kPOffLam);
-  float* gs = reinterpret_cast<float*>(sm + kPOffG);
-  float* cj = reinterpret_cast<float*>(sm + kPOffCj);
-  float* lamB = reinterpret_cast<float*>(sm + kPOffLamB);
-  float* scan = reinterpret_cast<float*>(sm + kPOffScan);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kPOffBar);
-  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kPOffMisc);  // [0] TMEM base, [1] abort
+  uint8_t* slots = sm + LY::kOffSlots;
+  uint8_t* qh = sm + LY::kOffQh;
+  float* lamA = reinterpret_cast<float*>(sm + LY::kOffLam);
+  float* gs = reinterpret_cast<float*>(sm + LY::kOffG);
+  float* cj = reinterpret_cast<float*>(sm + LY::kOffCj);
+  float* lamB = reinterpret_cast<float*>(sm + LY::kOffLamB);
+  float* scan = reinterpret_cast<float*>(sm + LY::kOffScan);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + LY::kOffBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + LY::kOffMisc);  // [0] TMEM base, [1] abort
   uint32_t* abort_flag = &misc[1];
 
   if (warp == 0) {
@@ -773,7 +786,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     // ------------------------------------------------------------ group A
     const int wa = warp - kPA0;     // 0..7
     const int part = wa >> 2;       // column blocks part, part + 2; K columns 32*part..
-    constexpr int kNP = (kLogC + 1 + kLevels) / 2;   // lam levels per thread: 0..13 over 2 parts
+    constexpr int kNP = (kLogC + 1 + kLevels + 1) / 2;   // lam levels per thread, over 2 parts
     float pf[kNP];
     float pf_la = 0.f;
     auto prefetch = [&](int c) {
@@ -848,8 +861,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       // start (g_row <= 0, so the factor stays finite)
       const float eg = __expf(g_row);
 #pragma unroll
-      for (int i = 4; i < kNP; ++i)
-        lamB[(gb * kC + row) * kLevels + part + 2 * i - (kLogC + 1)] = pfc[i] * eg;
+      for (int i = 4; i < kNP; ++i) {
+        const int b = part + 2 * i - (kLogC + 1);
+        if (b < kLevels) lamB[(gb * kC + row) * kLevels + b] = pfc[i] * eg;
+      }
       mbar_arrive(&bars[B_GREADY + gb]);
     };
     if (wa == 0 && lane == 0) l2_prefetch(1);
@@ -1025,7 +1040,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             mbar_arrive(&bars[B_REMPTY]);
             ++u;
           }
-          next_chain(c, b, cur0, cur1);
+          next_chain<NLEV>(c, b, cur0, cur1);
           W(B_RFULL, u & 1);
           tc_fence_after();
         }
@@ -1147,7 +1162,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile, va = qa + 2 * kTile;
         bool ok = true;
         int cb0 = 0, cb1 = 0;
-        for (bool more = next_chain(c, 0, cb0, cb1); more; more = next_chain(c, cb1 + 1, cb0, cb1)) {
+        for (bool more = next_chain<NLEV>(c, 0, cb0, cb1); more; more = next_chain<NLEV>(c, cb1 + 1, cb0, cb1)) {
           if ((c > 0 && !W(((c - 1) & 1) ? B_LV1 : B_LV, ((c - 1) >> 1) & 1)) ||
               !W(B_REMPTY, (u & 1) ^ 1)) {
             ok = false;
@@ -1239,14 +1254,22 @@ cudaError_t make_out_map(CUtensorMap* m, void* base, int H, long long tokens) {
 
 }  // namespace
 
+// The pipelined kernel keeps up to 7 chunk-level states on chip (T <= 16384); the serial
+// cross-check keeps 6 (T <= 8192).
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T) {
-  return in_dtype == LLATTN_BF16 && dk == kD && dv == kD && chunk == kC && T <= kC * kMaxChunks;
+  return in_dtype == LLATTN_BF16 && dk == kD && dv == kD && chunk == kC &&
+         T <= kC * (1 << PipeLong::kLev);
+}
+
+bool tc_serial_supports(int in_dtype, int dk, int dv, int chunk, int T) {
+  return tc_supports(in_dtype, dk, dv, chunk, T) && T <= kC * kMaxChunks;
 }
 
 size_t tc_workspace_bytes(int, int, int, int, int, int) { return 0; }
 
 cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool serial) {
-  if (!tc_supports(p.in_dtype, p.dk, p.dv, chunk, p.T)) return cudaErrorNotSupported;
+  if (!(serial ? tc_serial_supports : tc_supports)(p.in_dtype, p.dk, p.dv, chunk, p.T))
+    return cudaErrorNotSupported;
   // TMA only ever fetches whole chunks inside a sequence, so the token extent can be
   // the dense size, or for packed batches any bound >= the real total (nseq * T).
   const long long tokens = (long long)p.nseq * p.T;
@@ -1263,8 +1286,13 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
     if ((e = cudaFuncSetAttribute(tc_fwd_serial, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kSmemBytes)) != cudaSuccess)
       return e;
-    if ((e = cudaFuncSetAttribute(tc_fwd_pipe, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kPSmemBytes)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(tc_fwd_pipe<PipeShort::kLev, PipeShort::kSt>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PipeShort::kSmemBytes)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(tc_fwd_pipe<PipeLong::kLev, PipeLong::kSt>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PipeLong::kSmemBytes)) != cudaSuccess)
       return e;
     attr_set = true;
   }
@@ -1276,9 +1304,12 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
   if (serial)
     tc_fwd_serial<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, q, k, v, p.log_a, p.lam, p.out,
                                                       p.H, p.T, p.L, p.cu_seqlens, p.status);
-  else
-    tc_fwd_pipe<<<grid, kPThreads, kPSmemBytes, st>>>(mq, mk, mv, mo, q, k, v, p.log_a, p.lam, p.out,
-                                                      p.H, p.T, p.L, p.cu_seqlens, p.status);
+  else if (p.T <= kC * (1 << PipeShort::kLev))   // 6 levels on chip, three-stage ring
+    tc_fwd_pipe<PipeShort::kLev, PipeShort::kSt><<<grid, kPThreads, PipeShort::kSmemBytes, st>>>(
+        mq, mk, mv, mo, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens, p.status);
+  else                                            // 7 levels, two stages (shared memory)
+    tc_fwd_pipe<PipeLong::kLev, PipeLong::kSt><<<grid, kPThreads, PipeLong::kSmemBytes, st>>>(
+        mq, mk, mv, mo, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens, p.status);
   main_kernel_end(st);
   count_launch();
   return cudaGetLastError();

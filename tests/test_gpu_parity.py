@@ -23,12 +23,13 @@ W = I.WORKLOADS
 def _paths_for(inp):
     paths = ["simt"]
     if inp.dtype == "bf16":
-        try:
-            binding.workspace_bytes(1, "tcgen05", 0, inp.B, inp.H, inp.T, inp.dk, inp.dv,
-                                    inp.cu_seqlens is not None)
-            paths += ["tcgen05", "tcgen05_serial"]
-        except binding.LLAttnError:
-            pass
+        for path in ("tcgen05", "tcgen05_serial"):
+            try:
+                binding.workspace_bytes(1, path, 0, inp.B, inp.H, inp.T, inp.dk, inp.dv,
+                                        inp.cu_seqlens is not None)
+                paths.append(path)
+            except binding.LLAttnError:
+                pass
     return paths
 
 
@@ -51,6 +52,9 @@ CASES = {
     "t8k_d64_bf16_ragged": I.shrink(W["t8k_d64_bf16"], B=2, H=1, T=8000),
     "t64k_d128_bf16_t8k": I.shrink(W["t64k_d128_bf16"], H=2, T=8192),
     "varlen_small": I.shrink(W["varlen8_d64_bf16"], H=2, T=3000, len_lo=1, len_hi=3000),
+    # more than 64 chunks: the seventh chunk level and the two-stage variant of the kernel
+    "t12k_d64_bf16_h1": I.shrink(W["t8k_d64_bf16"], B=1, H=1, T=12000),
+    "varlen_long": I.shrink(W["varlen8_d64_bf16"], B=3, H=1, T=16384, len_lo=8000, len_hi=16384),
 }
 
 
@@ -70,6 +74,16 @@ def test_parity_workloads(name):
 def test_parity_decay_regimes(mode, base):
     w = I.shrink(W[base], B=1, H=2) if base == "t2k_d64_bf16" else W[base]
     inp = I.make_inputs(w, seed=1, log_a_mode=mode)
+    ref = O.llattn_recurrent(inp)
+    for path in _paths_for(inp):
+        _check(inp, ref, path)
+
+
+@pytest.mark.parametrize("level", [13, 14])
+def test_parity_one_hot_deep_level_long(level):
+    # level 14 reaches the seventh chunk-level state (blocks of 64 chunks): T > 8192, no decay
+    w = I.shrink(W["t8k_d64_bf16"], B=1, H=1, T=16384)
+    inp = I.make_inputs(w, seed=4, log_a_mode="zero", lam_mode="onehot", lam_level=level)
     ref = O.llattn_recurrent(inp)
     for path in _paths_for(inp):
         _check(inp, ref, path)
