@@ -79,7 +79,8 @@ enum { LLATTN_F32 = 0, LLATTN_BF16 = 1 };
 /* Kernel paths for llattn_fwd_ex.
  *   AUTO            tcgen05 path where one exists for the shape, else SIMT.
  *   SIMT            CUDA-core kernels (any dk, dv in {32,64,128}; fp32 or bf16 inputs).
- *   TCGEN05         tensor-core kernel, warp-specialised pipeline (bf16 inputs only; it
+ *   TCGEN05         tensor-core kernel, warp-specialised pipeline (bf16 inputs, d_k = d_v =
+ *                   64, chunk 128, T <= 16384; the serial cross-check T <= 8192; it
  *                   rounds P, V, the decay-scaled K and the level states once to fp16, so
  *                   those intermediates must stay below 6.5e4 in magnitude - true for
  *                   L2-normalised q, k and moderate v, lam; use SIMT otherwise).
