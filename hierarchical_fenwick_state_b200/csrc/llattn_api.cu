@@ -25,6 +25,8 @@ struct DeviceState {
   unsigned int* status = nullptr;
   void* stage = nullptr;  // llattn_fwd_host staging (inputs, output, cu_seqlens)
   size_t stage_bytes = 0;
+  cudaStream_t s_in = nullptr, s_out = nullptr;   // llattn_fwd_host copy streams
+  std::vector<cudaEvent_t> ev;                    // llattn_fwd_host ordering events
 };
 
 std::mutex g_mu;
@@ -399,6 +401,65 @@ llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const 
       {dv_, v, (size_t)total * H * dv * esz}, {da, log_a, (size_t)total * H * sizeof(float)},
       {dl, lam, (size_t)total * H * L * sizeof(float)},
       {dcu, cu_seqlens, (size_t)(B + 1) * sizeof(int)}};
+  if (cu_seqlens == nullptr && B >= 2) {
+    // Dense batch: each batch row is a contiguous slice of every tensor and an independent
+    // problem, so rows are pipelined - row b's upload (stream s_in), forward (the caller's
+    // stream) and download (stream s_out) overlap the other rows' copies in both directions.
+    if (ds->s_in == nullptr &&
+        (e = cudaStreamCreateWithFlags(&ds->s_in, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e);
+    if (ds->s_out == nullptr &&
+        (e = cudaStreamCreateWithFlags(&ds->s_out, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e);
+    const size_t nev = 2 * (size_t)B + 2;
+    while (ds->ev.size() < nev) {
+      cudaEvent_t x;
+      if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(e);
+      ds->ev.push_back(x);
+    }
+    cudaEvent_t* ev = ds->ev.data();   // [0] start, [1] done, [2 + 2b] uploaded, [3 + 2b] computed
+    const size_t rq = (size_t)T * H * dk * esz, rv = (size_t)T * H * dv * esz;
+    const size_t ra = (size_t)T * H * sizeof(float), rl = (size_t)T * H * L * sizeof(float);
+    const size_t ro = (size_t)T * H * dv * sizeof(float);
+    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ds->s_in, ev[0], 0)) != cudaSuccess)
+      return cuda_fail(e);
+    const char* hq = static_cast<const char*>(q);
+    const char* hk = static_cast<const char*>(k);
+    const char* hv = static_cast<const char*>(v);
+    const char* ha = reinterpret_cast<const char*>(log_a);
+    const char* hl = reinterpret_cast<const char*>(lam);
+    char* ho = reinterpret_cast<char*>(out);
+    for (int r = 0; r < B; ++r) {
+      const struct { char* d; const char* h; size_t n; } up[5] = {
+          {dq + r * rq, hq + r * rq, rq}, {dk_ + r * rq, hk + r * rq, rq},
+          {dv_ + r * rv, hv + r * rv, rv}, {reinterpret_cast<char*>(da) + r * ra, ha + r * ra, ra},
+          {reinterpret_cast<char*>(dl) + r * rl, hl + r * rl, rl}};
+      for (const auto& c : up)
+        if ((e = cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, ds->s_in)) != cudaSuccess)
+          return cuda_fail(e);
+      if ((e = cudaEventRecord(ev[2 + 2 * r], ds->s_in)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(st, ev[2 + 2 * r], 0)) != cudaSuccess)
+        return cuda_fail(e);
+      s = forward(in_dtype, LLATTN_PATH_AUTO, 0, dq + r * rq, dk_ + r * rq, dv_ + r * rv,
+                  reinterpret_cast<float*>(reinterpret_cast<char*>(da) + r * ra),
+                  reinterpret_cast<float*>(reinterpret_cast<char*>(dl) + r * rl),
+                  reinterpret_cast<float*>(reinterpret_cast<char*>(dout) + r * ro), 1, H, T, dk,
+                  dv, nullptr, nullptr, 0, stream);
+      if (s != LLATTN_OK) return s;
+      if ((e = cudaEventRecord(ev[3 + 2 * r], st)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(ds->s_out, ev[3 + 2 * r], 0)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(ho + r * ro, reinterpret_cast<char*>(dout) + r * ro, ro,
+                               cudaMemcpyDeviceToHost, ds->s_out)) != cudaSuccess)
+        return cuda_fail(e);
+    }
+    if ((e = cudaEventRecord(ev[1], ds->s_out)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(st, ev[1], 0)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+      return cuda_fail(e);
+    return LLATTN_OK;
+  }
   for (const auto& c : cp) {
     if (c.d == nullptr || c.n == 0) continue;
     if ((e = cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, st)) != cudaSuccess)

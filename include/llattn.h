@@ -167,6 +167,9 @@ LLATTN_API llattn_status llattn_device_status(unsigned int* flags, int clear);
  * (page-locked) for the copies to run at full speed.  in_dtype: LLATTN_BF16
  * (q, k, v as uint16 bf16 bit patterns) or LLATTN_F32.  cu_seqlens, if not NULL,
  * is a HOST int32 array [B+1]; the other arguments are as in llattn_fwd.
+ * Dense batches of two or more sequences are pipelined row by row: the upload of one
+ * row, the forward of another and the download of a third overlap (two copy streams
+ * the library keeps per device, ordered against `stream` with events).
  * Concurrent calls from several threads are serialised on an internal lock.
  */
 LLATTN_API llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const void* v,

@@ -184,3 +184,29 @@ def test_golden_fixtures(name, decay, dtype):
         sel = np.array([got[t, 0, j] for t, j, _ in rows])
         err = O.rel_max_err(sel, want)
         assert err <= TOL[dtype], f"{path}: rel max err {err:.3e}"
+
+
+# ------------------------------------------------------------------------------------------------
+# Host-buffer entry point (dense batches are pipelined row by row inside the library)
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["dense_pipelined", "dense_one_row", "varlen", "f32"])
+def test_host_entry_point_matches_device_path(name):
+    cases = {
+        "dense_pipelined": I.shrink(W["t2k_d64_bf16"], B=3, H=2, T=1000),
+        "dense_one_row": I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=700),
+        "varlen": I.shrink(W["varlen8_d64_bf16"], B=3, H=2, T=2000, len_lo=1, len_hi=2000),
+        "f32": I.shrink(W["t256_d32_f32"], B=2, T=250),
+    }
+    inp = I.make_inputs(cases[name], seed=9)
+    bf = inp.dtype == "bf16"
+    conv = (lambda x: np.ascontiguousarray(I.bf16_bits(x))) if bf else (lambda x: x)
+    out = np.full(inp.v.shape, np.nan, dtype=np.float32)
+    cu = np.ascontiguousarray(inp.cu_seqlens) if inp.cu_seqlens is not None else None
+    B = inp.B if cu is None else len(cu) - 1
+    binding.fwd_host(binding.BF16 if bf else binding.F32, conv(inp.q), conv(inp.k), conv(inp.v),
+                     inp.log_a, inp.lam, out, B, inp.H, inp.T, inp.dk, inp.dv, cu_seqlens=cu)
+    assert binding.device_status(clear=True) == 0
+    dev = run(inp, path="auto").astype(np.float32)
+    assert np.array_equal(out, dev), "host entry point differs from the device entry point"
+    err = O.rel_max_err(out.astype(np.float64), O.llattn_recurrent(inp))
+    assert err <= TOL[inp.dtype], f"rel max err {err:.3e}"
