@@ -797,7 +797,10 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 #pragma unroll
       for (int i = 0; i < kNP; ++i) {
         const int l = part + 2 * i;
-        pf[i] = (okt && l < L) ? __ldg(lr + l) : 0.f;
+        // inter-chunk levels only where chunk c reads them (bit l - 1 - log2 C of c): each
+        // row load that touches another cache sector costs the mask/scan warps time
+        const bool need = l <= kLogC || ((c >> (l - 1 - kLogC)) & 1);
+        pf[i] = (okt && l < L && need) ? __ldg(lr + l) : 0.f;
       }
       if (part == 0) pf_la = okt ? __ldg(log_a + tok * H + h) : 0.f;
     };
