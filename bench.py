@@ -81,11 +81,17 @@ def measured_peaks():
 
 
 def source_hash():
+    """Hash of the CUDA sources' code: comments and whitespace are left out, so that only a
+    change of the code itself makes a stored ncu capture stale."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_fenwick_state_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(name.encode() + " ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

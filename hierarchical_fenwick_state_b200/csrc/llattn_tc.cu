@@ -911,7 +911,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       W(B_SFULL, c & 1);
       tc_fence_after();
       named_sync(1, kPNA);  // cj and the lam table are visible to the whole group
-      // ---- causal Fenwick mask on S -> P (hi/lo), 16 keys at a time ----
+      // ---- causal Fenwick mask on S -> P (fp16, in place), 16 keys at a time ----
       // The two warps of a sub-partition take alternate 16-key groups, so each gets half of
       // the diagonal block (per-element levels) and half of every off-diagonal block.
       const uint32_t spc = tmem + lane_off + kPColSP;
@@ -970,7 +970,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       mbar_arrive(&bars[B_PFULL]);
       const float gend_c = gend;
       if (c + 1 < nch) decay_scan(c + 1);
-      // ---- chunk-state operand: K rows scaled by exp(G - g_s), hi in place, lo to klo ----
+      // ---- chunk-state operand: K rows scaled by exp(G - g_s), fp16, in place ----
       // (after the mask, overlapping P V(c) and S(c + 1) on the tensor cores).  The causal
       // mask loads sub-partitions 0..3 in the ratio 1:2:3:4, so the K rows are dealt out the
       // other way round: 48, 40, 24 and 16 rows to the two warps of sub-partitions 0..3.
