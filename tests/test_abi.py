@@ -77,3 +77,25 @@ def test_workspace_query():
     assert binding.workspace_bytes(1, "simt", 64, 0, 4, 1000, 64, 64, False) == 0
     with pytest.raises(binding.LLAttnError):
         binding.workspace_bytes(1, "simt", 64, 1, 4, 1000, 48, 64, False)
+
+
+def test_tensor_core_path_limits():
+    """The pipelined tensor-core kernel takes T <= 16384 (seven chunk levels on chip), the serial
+    cross-check T <= 8192; beyond that AUTO falls back to the CUDA-core path (no CUDA call)."""
+    ws = binding.workspace_bytes
+    for T in (1, 8192, 8193, 16384):
+        ws(binding.BF16, "tcgen05", 0, 2, 4, T, 64, 64, False)
+    ws(binding.BF16, "tcgen05_serial", 0, 2, 4, 8192, 64, 64, False)
+    for path, T in (("tcgen05", 16385), ("tcgen05_serial", 8193)):
+        with pytest.raises(binding.LLAttnError) as e:
+            ws(binding.BF16, path, 0, 2, 4, T, 64, 64, False)
+        assert e.value.status == 8   # LLATTN_ERR_UNSUPPORTED
+    for dk in (32, 128):             # the tensor-core kernel is built for d = 64
+        with pytest.raises(binding.LLAttnError):
+            ws(binding.BF16, "tcgen05", 0, 1, 1, 256, dk, dk, False)
+    with pytest.raises(binding.LLAttnError):   # bf16 inputs only
+        ws(binding.F32, "tcgen05", 0, 1, 1, 256, 64, 64, False)
+    # AUTO resolves without error for every supported shape (CUDA-core fallback beyond the limit)
+    for T in (16384, 16385, 65536):
+        ws(binding.BF16, "auto", 0, 1, 16, T, 64, 64, False)
+    ws(binding.BF16, "auto", 0, 1, 16, 65536, 128, 128, False)
