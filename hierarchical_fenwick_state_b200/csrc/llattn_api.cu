@@ -419,12 +419,20 @@ llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const 
       ds->ev.push_back(x);
     }
     cudaEvent_t* ev = ds->ev.data();   // [0] start, [1] done, [2 + 2b] uploaded, [3 + 2b] computed
+    // on a failure part-way, let the copies already queued finish before the staging memory
+    // can be reused by another call
+    auto drain = [&](llattn_status r) {
+      cudaStreamSynchronize(ds->s_in);
+      cudaStreamSynchronize(ds->s_out);
+      cudaStreamSynchronize(st);
+      return r;
+    };
     const size_t rq = (size_t)T * H * dk * esz, rv = (size_t)T * H * dv * esz;
     const size_t ra = (size_t)T * H * sizeof(float), rl = (size_t)T * H * L * sizeof(float);
     const size_t ro = (size_t)T * H * dv * sizeof(float);
     if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(ds->s_in, ev[0], 0)) != cudaSuccess)
-      return cuda_fail(e);
+      return drain(cuda_fail(e));
     const char* hq = static_cast<const char*>(q);
     const char* hk = static_cast<const char*>(k);
     const char* hv = static_cast<const char*>(v);
@@ -438,26 +446,26 @@ llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const 
           {reinterpret_cast<char*>(dl) + r * rl, hl + r * rl, rl}};
       for (const auto& c : up)
         if ((e = cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, ds->s_in)) != cudaSuccess)
-          return cuda_fail(e);
+          return drain(cuda_fail(e));
       if ((e = cudaEventRecord(ev[2 + 2 * r], ds->s_in)) != cudaSuccess ||
           (e = cudaStreamWaitEvent(st, ev[2 + 2 * r], 0)) != cudaSuccess)
-        return cuda_fail(e);
+        return drain(cuda_fail(e));
       s = forward(in_dtype, LLATTN_PATH_AUTO, 0, dq + r * rq, dk_ + r * rq, dv_ + r * rv,
                   reinterpret_cast<float*>(reinterpret_cast<char*>(da) + r * ra),
                   reinterpret_cast<float*>(reinterpret_cast<char*>(dl) + r * rl),
                   reinterpret_cast<float*>(reinterpret_cast<char*>(dout) + r * ro), 1, H, T, dk,
                   dv, nullptr, nullptr, 0, stream);
-      if (s != LLATTN_OK) return s;
+      if (s != LLATTN_OK) return drain(s);
       if ((e = cudaEventRecord(ev[3 + 2 * r], st)) != cudaSuccess ||
           (e = cudaStreamWaitEvent(ds->s_out, ev[3 + 2 * r], 0)) != cudaSuccess ||
           (e = cudaMemcpyAsync(ho + r * ro, reinterpret_cast<char*>(dout) + r * ro, ro,
                                cudaMemcpyDeviceToHost, ds->s_out)) != cudaSuccess)
-        return cuda_fail(e);
+        return drain(cuda_fail(e));
     }
     if ((e = cudaEventRecord(ev[1], ds->s_out)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(st, ev[1], 0)) != cudaSuccess ||
         (e = cudaStreamSynchronize(st)) != cudaSuccess)
-      return cuda_fail(e);
+      return drain(cuda_fail(e));
     return LLATTN_OK;
   }
   for (const auto& c : cp) {

@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/llattn.h"
@@ -1284,8 +1285,12 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
   if ((e = make_map(&mv, p.v, p.H, tokens)) != cudaSuccess) return e;
   CUtensorMap mo;
   if ((e = make_out_map(&mo, p.out, p.H, tokens)) != cudaSuccess) return e;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory opt-in is a per-device attribute of each kernel
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load()) {
     if ((e = cudaFuncSetAttribute(tc_fwd_serial, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kSmemBytes)) != cudaSuccess)
       return e;
@@ -1297,7 +1302,7 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)PipeLong::kSmemBytes)) != cudaSuccess)
       return e;
-    attr_set = true;
+    attr_set[dev].store(true);
   }
   const dim3 grid(p.H, p.nseq);
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
