@@ -261,3 +261,34 @@ def test_inputs_are_seeded_and_shaped():
     np.testing.assert_allclose(np.linalg.norm(a.q.astype(np.float64), axis=-1), 1.0, atol=1e-2)
     assert (a.log_a < 0).all() and (a.lam > 0).all()
     assert np.array_equal(I.round_to_bf16(a.v), a.v)
+
+
+# ----------------------------------------------------------------------------------------------
+# Limits with closed forms
+# ----------------------------------------------------------------------------------------------
+def test_strong_decay_limit_keeps_only_the_token_itself():
+    """With every gate a_t ~ 0 (log a = -60), every s < t is weighted by at most e^-60: the
+    output reduces to the level-0 term lam[t, 0] (q_t . k_t) v_t."""
+    inp = _rand_inputs(40, H=2, dk=5, dv=3, seed=11)
+    inp.log_a[...] = -60.0
+    q = inp.q.reshape(-1, inp.H, inp.dk).astype(np.float64)
+    k = inp.k.reshape(-1, inp.H, inp.dk).astype(np.float64)
+    v = inp.v.reshape(-1, inp.H, inp.dv).astype(np.float64)
+    lam0 = inp.lam.reshape(-1, inp.H, inp.L)[..., 0].astype(np.float64)
+    want = (lam0 * np.einsum("thd,thd->th", q, k))[..., None] * v
+    for form in (O.llattn_recurrent, O.llattn_quadratic):
+        got = form(inp).reshape(want.shape)
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-20)
+
+
+def test_two_token_closed_form():
+    """T = 2: o_0 = lam[0,0] (q0.k0) v0;  o_1 = lam[1,0] (q1.k1) v1 + lam[1,1] a_1 (q1.k0) v0."""
+    inp = _rand_inputs(2, H=1, dk=4, dv=3, seed=12)
+    q, k, v = (x.reshape(2, -1).astype(np.float64) for x in (inp.q, inp.k, inp.v))
+    lam = inp.lam.reshape(2, inp.L).astype(np.float64)
+    a1 = np.exp(np.float64(inp.log_a.reshape(2)[1]))
+    o0 = lam[0, 0] * (q[0] @ k[0]) * v[0]
+    o1 = lam[1, 0] * (q[1] @ k[1]) * v[1] + lam[1, 1] * a1 * (q[1] @ k[0]) * v[0]
+    for form in (O.llattn_bruteforce, O.llattn_quadratic, O.llattn_recurrent):
+        got = form(inp).reshape(2, -1)
+        np.testing.assert_allclose(got, np.stack([o0, o1]), rtol=1e-13, atol=0)
