@@ -210,3 +210,14 @@ def test_host_entry_point_matches_device_path(name):
     assert np.array_equal(out, dev), "host entry point differs from the device entry point"
     err = O.rel_max_err(out.astype(np.float64), O.llattn_recurrent(inp))
     assert err <= TOL[inp.dtype], f"rel max err {err:.3e}"
+
+
+@pytest.mark.parametrize("T", [8192, 8193, 16383])
+def test_kernel_boundaries_odd_heads(T):
+    # the last length of the six-level kernel, the first of the seven-level one, and a ragged
+    # tail at its limit; three heads (odd TMA head stride), two sequences
+    w = I.shrink(W["t8k_d64_bf16"], B=2, H=3, T=T)
+    inp = I.make_inputs(w, seed=T % 97, log_a_mode="slow")
+    ref = O.llattn_recurrent(inp)
+    for path in _paths_for(inp):
+        _check(inp, ref, path)
