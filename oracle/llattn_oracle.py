@@ -39,6 +39,11 @@ Forms (each cites the passage it follows):
     reduction checks (Spanish "Variantes Propuestas" item 1).
   * ``llattn_single``      - one output o_t by direct summation over s (the
     definition), for sampled checks at full size.
+  * ``llattn_decode_step`` - one token of the decoding form: gate the occupied
+    level states, read out, carry into the next level (section 2, "Forma
+    Ricorrente e Parallelizzata", decoding bullet); occupancy comes from the
+    position's bits alone.  ``llattn_level_states`` builds the states before a
+    position straight from the level definition, to start or check decoding.
 
 Parity status: every function here is pinned by tests that do not retype its
 formula (brute force on tiny inputs, Fenwick prefix decomposition, reduction
@@ -282,3 +287,110 @@ def rel_max_err(got, ref) -> float:
     if ref.size == 0:
         return 0.0
     return float(np.max(np.abs(got - ref)) / max(rms, 1e-300))
+
+
+# ----------------------------------------------------------------------------
+# Decoding form: one token per step over the O(log T) level states
+# ----------------------------------------------------------------------------
+def llattn_level_states(k, v, log_a, n: int, nslot: int):
+    """Level states of one sequence and head just before 0-based position n, from the definition.
+
+    Level l >= 1 holds the earlier tokens s < n with l(n, s) == l (the Fenwick bucket of
+    2**(l-1) tokens that exists iff bit l-1 of n is set; Log-Linear Attention, section 2,
+    "Partizionamento Gerarchico (Fenwick Tree)"), each as k_s v_s^T times the gate product
+    over r = s+1..n-1.  The gate of position n itself belongs to the step that reads the
+    states.  k [>= n, dk], v [>= n, dv], log_a [>= n] -> [nslot, dk, dv] for levels 1..nslot
+    (zero where the bucket is empty).
+    """
+    k = np.asarray(k, F64)[:n]
+    v = np.asarray(v, F64)[:n]
+    la = np.asarray(log_a, F64)[:n]
+    S = np.zeros((nslot, k.shape[1] if k.ndim == 2 else 0, v.shape[1] if v.ndim == 2 else 0), F64)
+    if n == 0:
+        return S
+    if n.bit_length() > nslot:
+        raise ValueError(f"position {n} needs {n.bit_length()} level slots, have {nslot}")
+    lev = fenwick_level_matrix(np.array([n]), np.arange(n))[0]
+    # sum_{r=s+1..n-1} log a_r for every s < n (0 for s = n-1)
+    suf = np.concatenate([np.cumsum(la[:0:-1])[::-1], [0.0]])
+    w = np.exp(suf)
+    for lvl in range(1, nslot + 1):
+        sel = lev == lvl
+        if sel.any():
+            S[lvl - 1] = (k[sel] * w[sel, None]).T @ v[sel]
+    return S
+
+
+def llattn_decode_step(S, n: int, q, k, v, log_a, lam):
+    """One step of the decoding (recurrent) form for one sequence and head at position n.
+
+    Log-Linear Attention, section 2, "Forma Ricorrente e Parallelizzata", decoding bullet:
+    the layer keeps one state per level of the hierarchy and each output is the per-level
+    weighted combination of those states; the Mamba-2 variant gates every state with the
+    scalar a_n (Spanish page, "Variantes Propuestas" item 1).
+
+    S [nslot, dk, dv]: the states of levels 1..nslot just before position n.  Which levels
+    hold a bucket is read off the binary counter n alone: level l is occupied iff bit l-1 of
+    n is set; the other slots are ignored, whatever they hold.  q, k [dk]; v [dv]; log_a and
+    lam[0 .. bit_length(n)] for this token.  Returns (o [dv], S_next), S_next being the states
+    just before position n + 1:
+      1. every occupied level is multiplied by a_n = exp(log_a);
+      2. the token's own state k v^T is level 0;
+      3. o = sum over level 0 and the occupied levels of lam[l] * (q^T S_l);
+      4. promotion (binary-counter carry): with m the number of trailing one bits of n,
+         levels 0..m add up into level m+1, and levels 1..m are emptied.  When m+1 > nslot,
+         position n is the last one the slots can hold and nothing is merged.
+    """
+    S = np.array(S, F64, copy=True)
+    nslot = S.shape[0]
+    if n < 0 or n.bit_length() > nslot:
+        raise ValueError(f"position {n} out of range for {nslot} level slots")
+    q = np.asarray(q, F64); k = np.asarray(k, F64); v = np.asarray(v, F64)
+    lam = np.asarray(lam, F64)
+    a = float(np.exp(np.float64(log_a)))
+    occupied = [lvl for lvl in range(1, nslot + 1) if (n >> (lvl - 1)) & 1]
+    for lvl in occupied:
+        S[lvl - 1] *= a
+    S0 = np.outer(k, v)
+    o = lam[0] * (q @ S0)
+    for lvl in occupied:
+        o = o + lam[lvl] * (q @ S[lvl - 1])
+    m = 0
+    while (n >> m) & 1:
+        m += 1
+    if m + 1 <= nslot:
+        merged = S0.copy()
+        for lvl in range(1, m + 1):
+            merged += S[lvl - 1]
+            S[lvl - 1] = 0.0
+        S[m] = merged
+    return o, S
+
+
+def llattn_decode_sequence(q, k, v, log_a, lam):
+    """One sequence and head decoded token by token from empty states: q,k [T,dk], v [T,dv],
+    log_a [T], lam [T,L] -> o [T,dv], with L - 1 level slots (levels 1..L-1)."""
+    q = np.asarray(q, F64)
+    T = q.shape[0]
+    lam = np.asarray(lam, F64)
+    nslot = lam.shape[1] - 1
+    S = np.zeros((nslot, q.shape[1], np.asarray(v).shape[1]), F64)
+    o = np.zeros((T, np.asarray(v).shape[1]), F64)
+    for n in range(T):
+        o[n], S = llattn_decode_step(S, n, q[n], k[n], v[n], log_a[n], lam[n])
+    return o
+
+
+def llattn_decode_batch(S, pos, q, k, v, log_a, lam):
+    """Decoding step over a batch: S [B,H,nslot,dk,dv] (states before each row's position),
+    pos [B] (tokens each row has absorbed), q,k [B,H,dk], v [B,H,dv], log_a [B,H],
+    lam [B,H,L] -> (o [B,H,dv], S_next)."""
+    S = np.asarray(S, F64)
+    B, H = S.shape[:2]
+    o = np.zeros((B, H, np.asarray(v).shape[2]), F64)
+    S_next = np.array(S, F64, copy=True)
+    for b in range(B):
+        for h in range(H):
+            o[b, h], S_next[b, h] = llattn_decode_step(S[b, h], int(pos[b]), q[b, h], k[b, h],
+                                                       v[b, h], log_a[b, h], lam[b, h])
+    return o, S_next
