@@ -80,13 +80,24 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
-def source_hash():
-    """Hash of the CUDA sources' code: comments and whitespace are left out, so that only a
-    change of the code itself makes a stored ncu capture stale."""
+# The CUDA sources each measured kernel is built from.  A stored ncu capture stays valid while
+# these files' code is unchanged; code elsewhere in the library (other kernels, the host API)
+# does not move that kernel's DRAM traffic.
+KERNEL_SOURCES = {
+    "tcgen05": ["llattn_tc.cu", "llattn_tc_ptx.cuh", "llattn_common.cuh", "llattn_internal.h"],
+    "simt": ["llattn_simt.cu", "llattn_common.cuh", "llattn_internal.h"],
+    "decode": ["llattn_decode.cu", "llattn_decode.h", "llattn_common.cuh"],
+}
+
+
+def source_hash(kernel_key):
+    """Hash of the code of the sources a kernel is built from (``kernel_key`` is
+    "<kernel>:<workload>"): comments and whitespace are left out, so that only a change of the
+    code itself makes a stored ncu capture stale."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_fenwick_state_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES[kernel_key.split(":")[0]]):
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -103,7 +114,7 @@ def ncu_traffic(kernel_key):
     with open(p) as f:
         d = json.load(f)
     ent = d.get(kernel_key)
-    if not ent or ent.get("source_hash") != source_hash():
+    if not ent or ent.get("source_hash") != source_hash(kernel_key):
         return None
     return ent.get("dram_bytes_per_launch")
 
