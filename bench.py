@@ -16,6 +16,10 @@ Prints ONE JSON line (rank 0) with the throughput, the dominant kernel's
 roofline fraction against the measured HBM bandwidth, the CPU oracle baseline,
 the end-to-end figure through the host-buffer C entry point, launch count and
 SM clocks sampled during the timed region.
+
+--workload decode_b64_h32_d64_bf16 times the decoding step instead: one new token for each of
+64 sequences whose positions are spread over [0, 8192), H=32, d=64, reading the level states
+the positions occupy and writing the carried one (tokens/s = sequences x steps / time).
 """
 from __future__ import annotations
 
@@ -71,6 +75,28 @@ def algorithmic_flops(w, lengths, chunk):
     return tot * w.H
 
 
+def decode_algorithmic_bytes(d):
+    """Bytes one decoding step must move, summed over (sequence, head): the occupied level
+    states read (popcount(n) of them), the carried state written (unless n is the last position
+    the slots hold), each slot's pending-gate scalar read and the new ones written, the token's
+    q, k, v, log_a and lam, and the fp32 output."""
+    esz = 2 if d.dtype == "bf16" else 4
+    nslot = d.L - 1
+    state = 4 * d.dk * d.dv
+    tot = 0
+    for n in (int(x) for x in d.pos):
+        occ = bin(n).count("1")
+        m = 0
+        while (n >> m) & 1:
+            m += 1
+        carry = 1 if m < nslot else 0
+        new_gates = bin((n + 1) & ((1 << nslot) - 1)).count("1")
+        per = (occ + carry) * state + 4 * (occ + new_gates) \
+            + (2 * d.dk + d.dv) * esz + 4 + 4 * d.L + 4 * d.dv
+        tot += per * d.H + 4   # + the position
+    return tot
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -86,7 +112,7 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "tcgen05": ["llattn_tc.cu", "llattn_tc_ptx.cuh", "llattn_common.cuh", "llattn_internal.h"],
     "simt": ["llattn_simt.cu", "llattn_common.cuh", "llattn_internal.h"],
-    "decode": ["llattn_decode.cu", "llattn_decode.h", "llattn_common.cuh"],
+    "decode": ["llattn_decode.cu", "llattn_decode.h", "llattn_common.cuh", "llattn_internal.h"],
 }
 
 
@@ -425,15 +451,228 @@ def run_ours(args, w, rank, world, local_rank):
     return line
 
 
+# ---------------------------------------------------------------------------------------------
+# decoding step
+# ---------------------------------------------------------------------------------------------
+DECODE_METRIC = "log-linear attn decode tokens/s, 64 sequences at positions < 8192, H=32, d=64 (1×B200)"
+
+
+def decode_config(w, d):
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv,
+            "positions": f"U[0, {1 << (w.L - 1)}) per sequence, seeded",
+            "inputs": f"{w.dtype} q/k/v, f32 log_a/lam, f32 out, f32 level states",
+            "state_bytes": int(d.B * d.H * (d.L - 1) * (d.dk * d.dv + 2) * 4),
+            "l2": "inputs larger than L2: each step reads "
+                  f"{decode_algorithmic_bytes(d) / 1e6:.0f} MB of level states (no flush)"}
+
+
+def oracle_decode_rate(d, pairs):
+    """Time the fp64 oracle's decoding step on `pairs` (sequence, head) pairs; tokens/s."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=1)
+    except Exception:  # noqa: BLE001
+        ctx = None
+    if ctx:
+        ctx.__enter__()
+    t0 = time.perf_counter()
+    for b, h in pairs:
+        O.llattn_decode_step(d.states[b, h], int(d.pos[b]), d.q[b, h], d.k[b, h], d.v[b, h],
+                             d.log_a[b, h], d.lam[b, h])
+    dt = time.perf_counter() - t0
+    if ctx:
+        ctx.__exit__(None, None, None)
+    rate = (len(pairs) / d.H) / dt
+    whole = "the whole step" if len(pairs) == d.B * d.H else f"a sample of {d.B * d.H}"
+    desc = (f"fp64 oracle decoding step on {len(pairs)} (sequence, head) pairs ({whole}), "
+            f"{dt:.2f} s, numpy single thread; tokens/s = pairs / H / time")
+    return rate, desc, dt
+
+
+def _decode_pairs(d, n):
+    import numpy as np
+    rng = np.random.default_rng(1)
+    return list(zip(rng.integers(0, d.B, n).tolist(), rng.integers(0, d.H, n).tolist()))
+
+
+def run_decode_reference(args, w, rank, world):
+    from hierarchical_fenwick_state_b200 import inputs as I
+    if rank != 0:
+        return None
+    d = I.make_decode_inputs(w, seed=args.seed)
+    pairs = _decode_pairs(d, 512)
+    for _ in range(args.warmup):
+        oracle_decode_rate(d, pairs[:64])
+    times, rates = [], []
+    for _ in range(args.steps):
+        r, desc, dt = oracle_decode_rate(d, pairs)
+        times.append(dt)
+        rates.append(r)
+    value = float(statistics.mean(rates))
+    return {
+        "metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": decode_config(w, d),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def run_decode(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from hierarchical_fenwick_state_b200 import binding
+    from hierarchical_fenwick_state_b200 import inputs as I
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    d = I.make_decode_inputs(w, seed=rank_seed(args.seed, rank))
+    B, H, L, dk, dv = d.B, d.H, d.L, d.dk, d.dv
+    dt = torch.bfloat16 if d.dtype == "bf16" else torch.float32
+    q = torch.from_numpy(d.q).to(dev).to(dt)
+    k = torch.from_numpy(d.k).to(dev).to(dt)
+    v = torch.from_numpy(d.v).to(dev).to(dt)
+    la = torch.from_numpy(d.log_a).to(dev)
+    lm = torch.from_numpy(d.lam).to(dev)
+    pos = torch.from_numpy(d.pos).to(dev)
+    nst = binding.decode_state_bytes(B, H, L, dk, dv) // 4
+    state = torch.empty(nst, dtype=torch.float32, device=dev)
+    nlev = B * H * (L - 1) * dk * dv
+    # each level stored without its pending gate, the gate row of the position's parity set
+    state[:nlev].view(B, H, L - 1, dk, dv).copy_(
+        torch.from_numpy(d.states * np.exp(-d.pending)[..., None, None]).to(dev))
+    gate = np.zeros((B, H, 2, L - 1), np.float32)
+    gate[np.arange(B), :, d.pos & 1] = d.pending
+    state[nlev:].copy_(torch.from_numpy(gate.reshape(-1)).to(dev))
+    out = torch.empty((B, H, dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # Re-running a step from the same positions reads the same slots and rewrites the same
+    # carried slot and gate row with the same values, so every timed step does the full work.
+    def step():
+        binding.decode_step(q, k, v, la, lm, pos, state, out, B, H, L, dk, dv)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    binding.profile_read(reset=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    binding.profile(True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    binding.profile(False)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    main_ms, main_n, launches = binding.profile_read(reset=True)
+    status = binding.device_status(clear=True)
+    if status:
+        raise RuntimeError(f"device status flags {status:#x} after the timed region")
+    ms_step = ms_total / args.steps
+    value = B * world / (ms_step / 1000.0)
+
+    hbm_gbs, _, peak_kind = measured_peaks()
+    abytes = decode_algorithmic_bytes(d)
+    main_avg_s = (main_ms / main_n) / 1000.0 if main_n else ms_step / 1000.0
+    kernel_key = f"decode:{w.name}"
+    roof = {"bound": "hbm", "achieved": abytes / main_avg_s / 1e9, "peak": hbm_gbs,
+            "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(kernel_key)
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "profiling-recipe fallback"
+    roof["kernel"] = kernel_key
+    roof["algorithmic_bytes_per_launch"] = abytes
+    roof["main_kernel_ms"] = main_avg_s * 1000.0
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if d.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": decode_config(w, d), "roofline": roof, "gpu_launches": launches,
+        "clocks": clk,
+    }
+
+    if not args.no_e2e:
+        # per step: this step's token inputs and positions up from pinned host memory, the step,
+        # the outputs back; the level states stay on the device between steps
+        if d.dtype == "bf16":
+            hq = torch.from_numpy(I.bf16_bits(d.q).view(np.int16)).pin_memory()
+            hk = torch.from_numpy(I.bf16_bits(d.k).view(np.int16)).pin_memory()
+            hv = torch.from_numpy(I.bf16_bits(d.v).view(np.int16)).pin_memory()
+        else:
+            hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (d.q, d.k, d.v))
+        hla = torch.from_numpy(d.log_a).pin_memory()
+        hlm = torch.from_numpy(d.lam).pin_memory()
+        hpos = torch.from_numpy(d.pos).pin_memory()
+        hout = torch.empty((B, H, dv), dtype=torch.float32).pin_memory()
+        dq, dk_, dv_ = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (hq, hk, hv))
+        dla, dlm, dpos = (torch.empty_like(x, device=dev) for x in (hla, hlm, hpos))
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hlm, hpos))
+        d2h = hout.numel() * 4
+
+        def e2e_step():
+            for dst, src in ((dq, hq), (dk_, hk), (dv_, hv), (dla, hla), (dlm, hlm), (dpos, hpos)):
+                dst.copy_(src, non_blocking=True)
+            binding.decode_step(dq, dk_, dv_, dla, dlm, dpos, state, out, B, H, L, dk, dv)
+            hout.copy_(out, non_blocking=True)
+            stream.synchronize()
+
+        for _ in range(3):
+            e2e_step()
+        n_e2e = max(10, min(args.steps, 100))
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1000.0 / n_e2e, dist, dev)
+        if not np.isfinite(hout.numpy()).all():
+            raise RuntimeError("non-finite decoding output")
+        line["e2e"] = {"value": B * world / e2e_s, "unit": "tokens/s",
+                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                       "steps": n_e2e,
+                       "entry": "llattn_decode_step, token inputs from pinned host memory"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, _ = oracle_decode_rate(d, [(b, h) for b in range(B) for h in range(H)])
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": desc}
+    return line
+
+
 def main():
     args = parse()
     from hierarchical_fenwick_state_b200 import inputs as I
-    w = I.WORKLOADS[args.workload]
+    decoding = args.workload in I.DECODE_WORKLOADS
+    w = I.DECODE_WORKLOADS[args.workload] if decoding else I.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        line = run_reference(args, w, rank, world)
+        line = (run_decode_reference if decoding else run_reference)(args, w, rank, world)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -446,7 +685,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, w, rank, world, local_rank)
+        line = (run_decode if decoding else run_ours)(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -22,7 +22,7 @@ EXPORTS = (
     "llattn_abi_version", "llattn_status_str", "llattn_num_levels", "llattn_fwd",
     "llattn_fwd_f32", "llattn_workspace_bytes", "llattn_fwd_ex", "llattn_device_status",
     "llattn_last_cuda_error", "llattn_fwd_host", "llattn_profile", "llattn_profile_read",
-    "llattn_fwd_noalloc",
+    "llattn_fwd_noalloc", "llattn_decode_state_bytes", "llattn_decode_step",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20  # LLATTN_NOALLOC_SCRATCH_BYTES
@@ -70,6 +70,10 @@ def lib():
     L.llattn_fwd_host.argtypes = [i, vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
     L.llattn_fwd_noalloc.restype = i
     L.llattn_fwd_noalloc.argtypes = [i, vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_decode_state_bytes.restype = i
+    L.llattn_decode_state_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+    L.llattn_decode_step.restype = i
+    L.llattn_decode_step.argtypes = [i, vp, vp, vp, f_p, f_p, i_p, f_p, f_p, i, i, i, i, i, vp]
     L.llattn_profile.restype = i
     L.llattn_profile.argtypes = [i]
     L.llattn_profile_read.restype = i
@@ -201,6 +205,32 @@ def fwd_noalloc(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None, stre
                                   ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None
                                   else None, _stream_handle(stream))
     _check(st, "llattn_fwd_noalloc")
+    return out
+
+
+def decode_state_bytes(B: int, H: int, L: int, dk: int, dv: int) -> int:
+    """Bytes of the decoding state buffer (llattn_decode_state_bytes)."""
+    n = ctypes.c_size_t(0)
+    _check(lib().llattn_decode_state_bytes(int(B), int(H), int(L), int(dk), int(dv),
+                                           ctypes.byref(n)), "llattn_decode_state_bytes")
+    return int(n.value)
+
+
+def decode_step(q, k, v, log_a, lam, pos, state, out, B, H, L, dk, dv, stream=None):
+    """Direct call of llattn_decode_step on raw device tensors: one new token per sequence.
+
+    q, k [B,H,dk] and v [B,H,dv] (bf16 or fp32), log_a [B,H] and lam [B,H,L] fp32, pos int32
+    [B] (tokens each sequence has absorbed; read only), state fp32 of decode_state_bytes()
+    bytes (kept between steps), out fp32 [B,H,dv]."""
+    in_dtype = BF16 if str(q.dtype) == "torch.bfloat16" else F32
+    st = lib().llattn_decode_step(in_dtype, ctypes.c_void_p(q.data_ptr()),
+                                  ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+                                  ctypes.c_void_p(log_a.data_ptr()),
+                                  ctypes.c_void_p(lam.data_ptr()), ctypes.c_void_p(pos.data_ptr()),
+                                  ctypes.c_void_p(state.data_ptr()),
+                                  ctypes.c_void_p(out.data_ptr()), int(B), int(H), int(L),
+                                  int(dk), int(dv), _stream_handle(stream))
+    _check(st, "llattn_decode_step")
     return out
 
 

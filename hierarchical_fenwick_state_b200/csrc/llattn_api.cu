@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "../../include/llattn.h"
+#include "llattn_decode.h"
 #include "llattn_internal.h"
 
 // Per-device status word: kernels OR LLATTN_DEV_* bits into it.
@@ -480,6 +481,48 @@ llattn_status llattn_fwd_host(int in_dtype, const void* q, const void* k, const 
                            cudaMemcpyDeviceToHost, st)) != cudaSuccess)
     return cuda_fail(e);
   if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_decode_state_bytes(int B, int H, int L, int dk, int dv, size_t* bytes) {
+  if (!bytes) return LLATTN_ERR_ARG;
+  if (B < 0 || H < 0 || B > 65535 || H > 65535 || L < 1 || L > 32) return LLATTN_ERR_SHAPE;
+  if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
+  *bytes = llattn::decode_state_bytes(B, H, L, dk, dv);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_decode_step(int in_dtype, const void* q, const void* k, const void* v,
+                                 const float* log_a, const float* lam, const int* pos,
+                                 float* state, float* out, int B, int H, int L, int dk, int dv,
+                                 void* stream) {
+  if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+  size_t state_bytes = 0;
+  llattn_status s = llattn_decode_state_bytes(B, H, L, dk, dv, &state_bytes);
+  if (s != LLATTN_OK) return s;
+  if (B == 0 || H == 0) return LLATTN_OK;  // nothing to compute
+  if (!q || !k || !v || !log_a || !lam || !pos || !state || !out) return LLATTN_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(state, 16) ||
+      !aligned(out, 16) || !aligned(log_a, 4) || !aligned(lam, 4) || !aligned(pos, 4))
+    return LLATTN_ERR_ALIGN;
+  // out must not overlap any input or the state
+  const size_t bh = (size_t)B * H, esz = in_dtype == LLATTN_BF16 ? 2 : 4;
+  const uintptr_t o0 = reinterpret_cast<uintptr_t>(out), o1 = o0 + bh * dv * sizeof(float);
+  const struct { const void* p; size_t n; } rng[7] = {
+      {q, bh * dk * esz}, {k, bh * dk * esz}, {v, bh * dv * esz}, {log_a, bh * sizeof(float)},
+      {lam, bh * L * sizeof(float)}, {pos, (size_t)B * sizeof(int)}, {state, state_bytes}};
+  for (const auto& r : rng) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(r.p), a1 = a0 + r.n;
+    if (r.n && a0 < o1 && o0 < a1) return LLATTN_ERR_ARG;
+  }
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  if ((s = device_state(&ds, &dev)) != LLATTN_OK) return s;
+  const size_t nlev = bh * (size_t)(L - 1) * dk * dv;
+  llattn::DecodeProblem p{in_dtype, q, k, v, log_a, lam, pos, state, state + nlev, out,
+                          B, H, L, dk, dv, ds->status};
+  const cudaError_t e = llattn::decode_step(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
   return LLATTN_OK;
 }
 

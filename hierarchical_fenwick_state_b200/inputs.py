@@ -241,3 +241,71 @@ def shrink(w: Workload, *, B: Optional[int] = None, H: Optional[int] = None,
         H=H if H is not None else w.H, T=T if T is not None else w.T,
         len_lo=len_lo if len_lo is not None else w.len_lo,
         len_hi=len_hi if len_hi is not None else w.len_hi)
+
+
+# ----------------------------------------------------------------------------
+# Decoding step inputs: one new token per sequence, level states from earlier tokens
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int        # sequences decoded together (one token each per step)
+    H: int
+    L: int        # levels; positions stay below 2**(L-1)
+    dk: int
+    dv: int
+    dtype: str    # "bf16" or "f32" for q/k/v
+    log_a_mu: float = -2.0
+
+
+# A serving-style batch: 64 sequences at positions spread over [0, 8192), H = 32, d = 64.
+DECODE_WORKLOADS = {
+    "decode_b64_h32_d64_bf16": DecodeWorkload("decode_b64_h32_d64_bf16", B=64, H=32, L=14,
+                                              dk=64, dv=64, dtype="bf16"),
+}
+
+
+@dataclasses.dataclass
+class DecodeInputs:
+    """Host arrays for one decoding step (fp32 storage; q/k/v bf16-exact for bf16)."""
+    q: np.ndarray          # [B, H, dk]
+    k: np.ndarray          # [B, H, dk]
+    v: np.ndarray          # [B, H, dv]
+    log_a: np.ndarray      # [B, H]
+    lam: np.ndarray        # [B, H, L]
+    pos: np.ndarray        # int32 [B]
+    states: np.ndarray     # [B, H, L-1, dk, dv]  level states before the step (every slot drawn)
+    pending: np.ndarray    # [B, H, L-1]  a draw in [-3, 0] per slot, for splitting a state
+    B: int
+    H: int
+    L: int
+    dk: int
+    dv: int
+    dtype: str
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: int = 0, *, positions=None) -> DecodeInputs:
+    """Draw one seeded decoding step.  Token inputs follow the forward's distributions; the
+    positions are uniform integers in [0, 2**(L-1)) unless given; the level states are
+    N(0, 0.3^2) per element (about the spread of a decayed sum of a few k v^T with unit k and
+    standard normal v), drawn for every slot, occupied or not."""
+    rng = np.random.default_rng(seed)
+    B, H, L, dk, dv = w.B, w.H, w.L, w.dk, w.dv
+    q = _l2_rows(rng.standard_normal((B, H, dk), dtype=np.float32))
+    k = _l2_rows(rng.standard_normal((B, H, dk), dtype=np.float32))
+    v = rng.standard_normal((B, H, dv), dtype=np.float32)
+    log_a = -np.exp(w.log_a_mu + 0.5 * rng.standard_normal((B, H), dtype=np.float32))
+    lam = _softplus(rng.standard_normal((B, H, L), dtype=np.float32))
+    if positions is None:
+        pos = rng.integers(0, 1 << (L - 1), size=B)
+    else:
+        pos = np.asarray(positions)
+        assert pos.shape == (B,)
+    states = 0.3 * rng.standard_normal((B, H, L - 1, dk, dv), dtype=np.float32)
+    pending = -3.0 * rng.random((B, H, L - 1), dtype=np.float32)
+    if w.dtype == "bf16":
+        q, k, v = round_to_bf16(q), round_to_bf16(k), round_to_bf16(v)
+    f = lambda x: np.ascontiguousarray(x, np.float32)  # noqa: E731
+    return DecodeInputs(q=f(q), k=f(k), v=f(v), log_a=f(log_a), lam=f(lam),
+                        pos=np.ascontiguousarray(pos, np.int32), states=f(states),
+                        pending=f(pending), B=B, H=H, L=L, dk=dk, dv=dv, dtype=w.dtype)

@@ -97,7 +97,8 @@ enum {
 enum {
   LLATTN_DEV_SEQ_TOO_LONG = 1u,  /* a varlen sequence was longer than T */
   LLATTN_DEV_WAIT_TIMEOUT = 2u,  /* an mbarrier / pipeline wait hit its iteration limit */
-  LLATTN_DEV_BAD_CU_SEQLENS = 4u /* cu_seqlens decreasing */
+  LLATTN_DEV_BAD_CU_SEQLENS = 4u, /* cu_seqlens decreasing */
+  LLATTN_DEV_DECODE_POS = 8u     /* llattn_decode_step: a position outside [0, 2^(L-1)) */
 };
 
 /* Version of this ABI (increments on any signature change). */
@@ -223,6 +224,56 @@ LLATTN_API llattn_status llattn_fwd_noalloc(int in_dtype, const void* q, const v
                                             const void* v, const float* log_a, const float* lam,
                                             float* out, int B, int H, int T, int dk, int dv,
                                             const int* cu_seqlens, void* stream);
+
+/*
+ * Decoding: one new token per sequence per call, over the O(log T) level states.
+ *
+ * Log-Linear Attention (gist.science summaries, Italian "Sommario tecnico" section 2, "Forma
+ * Ricorrente e Parallelizzata", decoding bullet; Spanish "Resumen tecnico" section 2,
+ * "Particion Jerarquica"): at inference the layer keeps one d_k x d_v state per Fenwick
+ * level and combines them with the per-level weights.  For the token at 0-based position n
+ * of a sequence, with Mamba-2's scalar gate a_n = exp(log_a):
+ *   1. every occupied level l >= 1 is gated by a_n; level 0 is k_n v_n^T;
+ *   2. o_n = sum over level 0 and the occupied levels l of lam[l] * (q_n^T S_l);
+ *   3. with m the number of trailing one bits of n, levels 0..m are summed into level m+1
+ *      and levels 1..m fall empty (a binary-counter carry).
+ * Level l >= 1 is occupied exactly when bit l-1 of n is set, so a sequence's position is its
+ * whole occupancy record.  Decoding tokens 0..T-1 of a sequence this way gives the outputs
+ * llattn_fwd gives for that sequence (same operation, one token at a time).
+ *
+ * llattn_decode_state_bytes - size of the state buffer of B sequences x H heads whose
+ * positions stay below 2^(L-1) (L = llattn_num_levels(T) for sequences of at most T tokens):
+ * B*H*(L-1)*dk*dv*4 + B*H*2*(L-1)*4 bytes.  1 <= L <= 32.
+ *
+ * llattn_decode_step - one step for every sequence of the batch.
+ *   in_dtype  LLATTN_BF16 (q, k, v as uint16 bf16 bit patterns) or LLATTN_F32.
+ *   q, k      [B, H, dk]; v [B, H, dv]: each sequence's new token.  log_a [B, H] fp32;
+ *             lam [B, H, L] fp32 (level innermost; entries above the position's highest
+ *             level are read but unused).  out [B, H, dv] fp32, fully overwritten.
+ *   pos       DEVICE int32 [B]: tokens sequence b has absorbed, i.e. the new token's position.
+ *             Read only: the caller advances it for the next step.  Setting pos[b] = 0 starts
+ *             sequence b afresh; nothing else in the state has to be reset or cleared.
+ *   state     DEVICE fp32 buffer of llattn_decode_state_bytes(), caller-owned and kept
+ *             between steps.  Layout: levels [B, H, L-1, dk, dv] (slot j = level j+1, row-major
+ *             dk x dv), then gate [B, H, 2, L-1].  A slot holds its level's state as it was
+ *             when written; gate[b, h, p, j] is the log of the gate product slot j has missed
+ *             since then, valid at positions of parity p.  The level's state just before
+ *             position n is exp(gate[b, h, n & 1, j]) * levels[b, h, j].  To start from states
+ *             computed elsewhere, write them to levels with gate[b, h, pos[b] & 1, :] = 0.
+ *   dk, dv    in {32, 64, 128}.  B, H <= 65535.
+ * Pointers: q, k, v, state and out 16-byte aligned, log_a, lam and pos 4-byte aligned; out
+ * must not overlap the inputs or the state.  Asynchronous on `stream`.  A position outside
+ * [0, 2^(L-1)) leaves that sequence's output and state untouched and sets
+ * LLATTN_DEV_DECODE_POS in the device status word.  Steps that share a state buffer must run
+ * in order (one stream); arithmetic is fp32 on CUDA cores (an HBM-bound step: it reads each
+ * occupied level state once and writes the carried one).
+ */
+LLATTN_API llattn_status llattn_decode_state_bytes(int B, int H, int L, int dk, int dv,
+                                                   size_t* bytes);
+LLATTN_API llattn_status llattn_decode_step(int in_dtype, const void* q, const void* k,
+                                            const void* v, const float* log_a, const float* lam,
+                                            const int* pos, float* state, float* out, int B,
+                                            int H, int L, int dk, int dv, void* stream);
 
 /*
  * Launch accounting, for benchmarks.  llattn_profile(1) starts recording a pair

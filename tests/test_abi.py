@@ -99,3 +99,42 @@ def test_tensor_core_path_limits():
     for T in (16384, 16385, 65536):
         ws(binding.BF16, "auto", 0, 1, 16, T, 64, 64, False)
     ws(binding.BF16, "auto", 0, 1, 16, 65536, 128, 128, False)
+
+
+def _decode(**kw):
+    a = dict(in_dtype=1, q=0x1000, k=0x2000, v=0x3000, log_a=0x4000, lam=0x5000, pos=0x5800,
+             state=0x10000, out=0x8000, B=2, H=3, L=14, dk=64, dv=64)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return binding.lib().llattn_decode_step(a["in_dtype"], vp(a["q"]), vp(a["k"]), vp(a["v"]),
+                                            vp(a["log_a"]), vp(a["lam"]), vp(a["pos"]),
+                                            vp(a["state"]), vp(a["out"]), a["B"], a["H"], a["L"],
+                                            a["dk"], a["dv"], None)
+
+
+def test_decode_state_bytes():
+    for B, H, L, dk, dv in ((1, 1, 1, 32, 32), (64, 32, 14, 64, 64), (3, 5, 17, 128, 32)):
+        assert binding.decode_state_bytes(B, H, L, dk, dv) == \
+            B * H * (L - 1) * dk * dv * 4 + B * H * 2 * (L - 1) * 4
+    for bad in ((1, 1, 0, 64, 64), (1, 1, 33, 64, 64), (1, 1, 14, 48, 64), (-1, 1, 14, 64, 64),
+                (65536, 1, 14, 64, 64)):
+        with pytest.raises(binding.LLAttnError) as e:
+            binding.decode_state_bytes(*bad)
+        assert e.value.status == 2
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48), 2), (dict(dv=256), 2), (dict(L=0), 2), (dict(L=33), 2), (dict(B=-1), 2),
+    (dict(in_dtype=5), 4),
+    (dict(q=0), 1), (dict(pos=0), 1), (dict(state=0), 1),
+    (dict(q=0x1008), 3), (dict(state=0x10004), 3), (dict(out=0x8008), 3), (dict(pos=0x5802), 3),
+    # out overlaps the state (state starts at 0x10000) or lam (6 rows x 14 levels x 4 B at 0x5000)
+    (dict(out=0x10100), 1), (dict(out=0x5010), 1),
+])
+def test_decode_argument_errors_before_launch(kw, status):
+    assert _decode(**kw) == status
+
+
+def test_decode_empty_batches_are_no_ops():
+    assert _decode(B=0) == 0
+    assert _decode(H=0) == 0
