@@ -44,6 +44,8 @@ Forms (each cites the passage it follows):
     Ricorrente e Parallelizzata", decoding bullet); occupancy comes from the
     position's bits alone.  ``llattn_level_states`` builds the states before a
     position straight from the level definition, to start or check decoding.
+  * ``llattn_backward``    - gradients of sum(do * o) with respect to q, k, v,
+    log_a and lam, by differentiating the masked form product by product.
 
 Parity status: every function here is pinned by tests that do not retype its
 formula (brute force on tiny inputs, Fenwick prefix decomposition, reduction
@@ -394,3 +396,79 @@ def llattn_decode_batch(S, pos, q, k, v, log_a, lam):
             o[b, h], S_next[b, h] = llattn_decode_step(S[b, h], int(pos[b]), q[b, h], k[b, h],
                                                        v[b, h], log_a[b, h], lam[b, h])
     return o, S_next
+
+
+# ----------------------------------------------------------------------------
+# Backward: gradients of the masked (parallel) form
+# ----------------------------------------------------------------------------
+def llattn_backward_seq(q, k, v, log_a, lam, do):
+    """Gradients of sum(do * o) for one sequence and head, o = ((Q K^T) .* M_H) V.
+
+    The forward is the parallel form of Log-Linear Attention (section 2, "Matrici
+    Gerarchiche"; Spanish "Forma Paralela para Entrenamiento"): A = Q K^T, M[t, s] =
+    lam[t, l(t, s)] * exp(g_t - g_s) for s <= t, P = A .* M, O = P V, with g the
+    inclusive cumulative sum of log_a.  Differentiating each product in turn:
+      dV = P^T dO;   dP = dO V^T;   dQ = (dP .* M) K;   dK = (dP .* M)^T Q;
+      dM = dP .* A   (on s <= t);
+      dlam[t, l] = sum over s <= t with l(t, s) == l of dM[t, s] * exp(g_t - g_s);
+      dE = dM .* M   (the gradient of the exponent g_t - g_s);
+      dg_t = sum_s dE[t, s] - sum_t' dE[t', t];
+      dlog_a[r] = sum over t >= r of dg_t   (g_t sums log_a over positions <= t).
+    Inputs q,k [T,dk]; v, do [T,dv]; log_a [T]; lam [T,L].  Returns fp64
+    (dq, dk, dv, dlog_a, dlam).
+    """
+    q = np.asarray(q, F64); k = np.asarray(k, F64); v = np.asarray(v, F64)
+    do = np.asarray(do, F64)
+    g = np.cumsum(np.asarray(log_a, F64))
+    lam = np.asarray(lam, F64)
+    T = q.shape[0]
+    L = lam.shape[1]
+    tt = np.arange(T)
+    lev = fenwick_level_matrix(tt, tt)
+    causal = tt[None, :] <= tt[:, None]
+    E = np.where(causal, np.exp(np.where(causal, g[:, None] - g[None, :], 0.0)), 0.0)
+    lam_sel = np.take_along_axis(lam, np.where(causal, lev, 0), axis=1)
+    M = np.where(causal, lam_sel * E, 0.0)
+    A = q @ k.T
+    P = A * M
+    dv = P.T @ do
+    dP = do @ v.T
+    dA = dP * M
+    dq = dA @ k
+    dk = dA.T @ q
+    dM = np.where(causal, dP * A, 0.0)
+    dlam = np.zeros((T, L), F64)
+    contrib = dM * E
+    for lvl in range(L):
+        dlam[:, lvl] = np.sum(np.where(causal & (lev == lvl), contrib, 0.0), axis=1)
+    dE = dM * M
+    dg = dE.sum(axis=1) - dE.sum(axis=0)
+    dlog_a = np.cumsum(dg[::-1])[::-1]
+    return dq, dk, dv, dlog_a, dlam
+
+
+def llattn_backward(inp, do):
+    """Whole-input gradients (dense or packed), fp64, laid out like the inputs:
+    returns dict q, k, v, log_a, lam.  do has the layout of the output."""
+    H = inp.H
+    res = {
+        "q": np.zeros(inp.q.reshape(-1, H, inp.dk).shape, F64),
+        "k": np.zeros(inp.k.reshape(-1, H, inp.dk).shape, F64),
+        "v": np.zeros(inp.v.reshape(-1, H, inp.dv).shape, F64),
+        "log_a": np.zeros(inp.log_a.reshape(-1, H).shape, F64),
+        "lam": np.zeros(inp.lam.reshape(-1, H, inp.L).shape, F64),
+    }
+    dof = np.asarray(do).reshape(-1, H, inp.dv)
+    for sl, q, k, v, la, lm in _per_sequence(inp):
+        if q.shape[1] == 0:
+            continue
+        for h in range(H):
+            dq, dk, dv, dla, dlm = llattn_backward_seq(q[h], k[h], v[h], la[h], lm[h], dof[sl, h])
+            res["q"][sl, h] = dq
+            res["k"][sl, h] = dk
+            res["v"][sl, h] = dv
+            res["log_a"][sl, h] = dla
+            res["lam"][sl, h] = dlm
+    return {"q": res["q"].reshape(inp.q.shape), "k": res["k"].reshape(inp.k.shape),
+            "v": res["v"].reshape(inp.v.shape), "log_a": res["log_a"].reshape(inp.log_a.shape),
+            "lam": res["lam"].reshape(inp.lam.shape)}
