@@ -17,6 +17,9 @@ roofline fraction against the measured HBM bandwidth, the CPU oracle baseline,
 the end-to-end figure through the host-buffer C entry point, launch count and
 SM clocks sampled during the timed region.
 
+--pass bwd times the backward pass over the same workload: dq, dk, dv, dlog_a and dlam from
+q, k, v, log_a, lam and the output gradient (tokens/s of gradient computation).
+
 --workload decode_b64_h32_d64_bf16 times the decoding step instead: one new token for each of
 64 sequences whose positions are spread over [0, 8192), H=32, d=64, reading the level states
 the positions occupy and writing the carried one (tokens/s = sequences x steps / time).
@@ -50,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd times the backward pass (gradients of all inputs) instead")
     return ap.parse_args()
 
 
@@ -97,6 +102,36 @@ def decode_algorithmic_bytes(d):
     return tot
 
 
+def bwd_algorithmic(w, lengths):
+    """Bytes and FLOPs of one backward step.  Bytes: read q, k, v, dout (input type), log_a, lam;
+    write dq, dk, dv, dlog_a, dlam (fp32).  FLOPs of the level-by-level form: every causal pair
+    inside an aligned 32-token tile costs two dot products and three product terms (10 d); at
+    each level l >= 6, every token of a block with both halves present adds its outer product
+    to a d x d state (2 d^2) and applies the other half's state (2 d^2 on the right half,
+    4 d^2 on the left)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    d = w.dk
+    per = (2 * w.dk + 2 * w.dv) * esz + 4 + 4 * w.L + (2 * w.dk + w.dv) * 4 + 4 + 4 * w.L
+    flops = 0
+    for n in lengths:
+        for t0 in range(0, n, 32):
+            m = min(32, n - t0)
+            flops += m * (m + 1) // 2 * 10 * d
+        for lvl in range(6, w.L):
+            half = 1 << (lvl - 1)
+            for lo in range(0, n, 2 * half):
+                nl = min(half, n - lo)
+                nr = max(0, min(2 * half, n - lo) - half)
+                if nr:
+                    flops += (nl + nr) * 2 * d * d + nr * 2 * d * d + nl * 4 * d * d
+    return per * sum(lengths) * w.H, flops * w.H, per
+
+
+def alu_peak_tflops():
+    """fp32 FMA peak of a B200: 148 SMs x 128 fp32 lanes x 2 FLOPs x 1965 MHz (max SM clock)."""
+    return 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -113,6 +148,7 @@ KERNEL_SOURCES = {
     "tcgen05": ["llattn_tc.cu", "llattn_tc_ptx.cuh", "llattn_common.cuh", "llattn_internal.h"],
     "simt": ["llattn_simt.cu", "llattn_common.cuh", "llattn_internal.h"],
     "decode": ["llattn_decode.cu", "llattn_decode.h", "llattn_common.cuh", "llattn_internal.h"],
+    "bwd": ["llattn_bwd.cu", "llattn_bwd.h", "llattn_common.cuh", "llattn_internal.h"],
 }
 
 
@@ -663,6 +699,228 @@ def run_decode(args, w, rank, world, local_rank):
     return line
 
 
+# ---------------------------------------------------------------------------------------------
+# backward pass
+# ---------------------------------------------------------------------------------------------
+BWD_METRIC = "log-linear attn bwd tokens/s at T=8K,H=32,d=64 (1×B200)"
+
+
+def oracle_bwd_rate(inp, do, n_pairs):
+    """Time the oracle's direct-sum gradients (dq, dk, dv, dlam rows and columns) on n_pairs
+    (token, head) pairs; tokens/s of gradient rows = pairs / H / time."""
+    import numpy as np
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=1)
+    except Exception:  # noqa: BLE001
+        ctx = None
+    rng = np.random.default_rng(1)
+    total = inp.total_tokens
+    samples = list(zip(rng.integers(0, total, n_pairs).tolist(),
+                       rng.integers(0, inp.H, n_pairs).tolist()))
+    if ctx:
+        ctx.__enter__()
+    t0 = time.perf_counter()
+    O.llattn_backward_sampled(inp, do, samples)
+    dt = time.perf_counter() - t0
+    if ctx:
+        ctx.__exit__(None, None, None)
+    desc = (f"fp64 oracle, direct sums of the dq, dk, dv and dlam rows of {n_pairs} sampled "
+            f"(token, head) pairs (dlog_a not included), {dt:.2f} s, numpy single thread; "
+            f"tokens/s = pairs / H / time")
+    return (n_pairs / inp.H) / dt, desc, dt
+
+
+def bwd_config(w, path):
+    cfg = workload_config(w, None, path)
+    cfg["pass"] = "bwd"
+    cfg["inputs"] = f"{w.dtype} q/k/v/dout (dout ~ N(0,1)), f32 log_a/lam, f32 gradients"
+    return cfg
+
+
+def _bwd_do(inp, seed):
+    import numpy as np
+    from hierarchical_fenwick_state_b200 import inputs as I
+    do = np.random.default_rng(seed + 1000).standard_normal(inp.v.shape).astype(np.float32)
+    return I.round_to_bf16(do) if inp.dtype == "bf16" else do
+
+
+def run_bwd_reference(args, w, rank, world):
+    from hierarchical_fenwick_state_b200 import inputs as I
+    if rank != 0:
+        return None
+    inp = I.make_inputs(w, seed=args.seed)
+    do = _bwd_do(inp, args.seed)
+    for _ in range(args.warmup):
+        oracle_bwd_rate(inp, do, 32)
+    times, rates = [], []
+    for _ in range(args.steps):
+        r, desc, dt = oracle_bwd_rate(inp, do, 256)
+        times.append(dt)
+        rates.append(r)
+    value = float(statistics.mean(rates))
+    return {
+        "metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": bwd_config(w, None),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def run_bwd(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from hierarchical_fenwick_state_b200 import binding
+    from hierarchical_fenwick_state_b200 import inputs as I
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    inp = I.make_inputs(w, seed=rank_seed(args.seed, rank))
+    do = _bwd_do(inp, rank_seed(args.seed, rank))
+    dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    names = ("q", "k", "v", "log_a", "lam")
+    x = {n: torch.from_numpy(getattr(inp, n)).to(dev) for n in names}
+    for n in ("q", "k", "v"):
+        x[n] = x[n].to(dt)
+    tdo = torch.from_numpy(do).to(dev).to(dt)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev) if inp.cu_seqlens is not None else None
+    grads = {n: torch.empty(getattr(inp, n).shape, dtype=torch.float32, device=dev) for n in names}
+    nws = binding.bwd_workspace_bytes(inp.B, inp.H, inp.T, inp.dk, inp.dv)
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    lengths = [n for _, n in inp.seq_slices()]
+    total_tokens = int(sum(lengths))
+
+    def step():
+        binding.backward(x["q"], x["k"], x["v"], x["log_a"], x["lam"], tdo, cu_seqlens=cu,
+                         T=inp.T, grads=grads, workspace=ws)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    binding.profile_read(reset=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    binding.profile(True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    binding.profile(False)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    main_ms, main_n, launches = binding.profile_read(reset=True)
+    status = binding.device_status(clear=True)
+    if status:
+        raise RuntimeError(f"device status flags {status:#x} after the timed region")
+    ms_step = ms_total / args.steps
+    value = total_tokens * world / (ms_step / 1000.0)
+
+    hbm_gbs, _, peak_kind = measured_peaks()
+    abytes, aflops, per_tok = bwd_algorithmic(w, lengths)
+    alu = alu_peak_tflops()
+    main_avg_s = (main_ms / main_n) / 1000.0 if main_n else ms_step / 1000.0
+    kernel_key = f"bwd:{w.name}"
+    if aflops / (alu * 1e12) >= abytes / (hbm_gbs * 1e9):
+        roof = {"bound": "alu", "achieved": aflops / main_avg_s / 1e12, "peak": alu,
+                "unit": "TFLOP/s",
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz (fp32 FMA)"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / main_avg_s / 1e9, "peak": hbm_gbs,
+                "unit": "GB/s", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(kernel_key)
+    roof["kernel"] = kernel_key + " (all backward kernels of one call, one event pair)"
+    roof["algorithmic_bytes_per_launch"] = abytes
+    roof["algorithmic_flops_per_launch"] = aflops
+    roof["hbm_frac"] = abytes / main_avg_s / 1e9 / hbm_gbs
+    roof["bytes_per_token_head"] = per_tok
+    roof["main_kernel_ms"] = main_avg_s * 1000.0
+    line = {
+        "metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": bwd_config(w, "simt level-by-level"),
+        "roofline": roof, "gpu_launches": launches, "clocks": clk,
+    }
+
+    if not args.no_e2e:
+        # inputs and the output gradient up from pinned host memory, the backward, all five
+        # gradients back, every step
+        hx = {}
+        for n in names:
+            a = getattr(inp, n)
+            if n in ("q", "k", "v") and inp.dtype == "bf16":
+                hx[n] = torch.from_numpy(I.bf16_bits(a).view(np.int16)).pin_memory()
+            else:
+                hx[n] = torch.from_numpy(a).pin_memory()
+        hdo = (torch.from_numpy(I.bf16_bits(do).view(np.int16)) if inp.dtype == "bf16"
+               else torch.from_numpy(do)).pin_memory()
+        hg = {n: torch.empty(getattr(inp, n).shape, dtype=torch.float32).pin_memory()
+              for n in names}
+        dx = {n: torch.empty(hx[n].shape, dtype=hx[n].dtype, device=dev) for n in names}
+        ddo = torch.empty(hdo.shape, dtype=hdo.dtype, device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in list(hx.values()) + [hdo])
+        d2h = sum(t.numel() * 4 for t in hg.values())
+
+        def e2e_step():
+            for n in names:
+                dx[n].copy_(hx[n], non_blocking=True)
+            ddo.copy_(hdo, non_blocking=True)
+            qv = {n: (dx[n].view(torch.bfloat16) if n in ("q", "k", "v") and inp.dtype == "bf16"
+                      else dx[n]) for n in names}
+            binding.backward(qv["q"], qv["k"], qv["v"], qv["log_a"], qv["lam"],
+                             ddo.view(torch.bfloat16) if inp.dtype == "bf16" else ddo,
+                             cu_seqlens=cu, T=inp.T, grads=grads, workspace=ws)
+            for n in names:
+                hg[n].copy_(grads[n], non_blocking=True)
+            stream.synchronize()
+
+        for _ in range(2):
+            e2e_step()
+        n_e2e = max(3, min(args.steps, 10))
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1000.0 / n_e2e, dist, dev)
+        if not all(np.isfinite(hg[n].numpy()).all() for n in names):
+            raise RuntimeError("non-finite gradients through the host copies")
+        line["e2e"] = {"value": total_tokens * world / e2e_s, "unit": "tokens/s",
+                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                       "steps": n_e2e, "entry": "llattn_bwd, inputs and gradients through pinned "
+                                                "host memory"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, _ = oracle_bwd_rate(inp, do, 1024)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": desc}
+    return line
+
+
 def main():
     args = parse()
     from hierarchical_fenwick_state_b200 import inputs as I
@@ -672,7 +930,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        line = (run_decode_reference if decoding else run_reference)(args, w, rank, world)
+        if args.which == "bwd" and not decoding:
+            line = run_bwd_reference(args, w, rank, world)
+        else:
+            line = (run_decode_reference if decoding else run_reference)(args, w, rank, world)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -685,7 +946,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = (run_decode if decoding else run_ours)(args, w, rank, world, local_rank)
+        if args.which == "bwd" and not decoding:
+            line = run_bwd(args, w, rank, world, local_rank)
+        else:
+            line = (run_decode if decoding else run_ours)(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -23,6 +23,7 @@ EXPORTS = (
     "llattn_fwd_f32", "llattn_workspace_bytes", "llattn_fwd_ex", "llattn_device_status",
     "llattn_last_cuda_error", "llattn_fwd_host", "llattn_profile", "llattn_profile_read",
     "llattn_fwd_noalloc", "llattn_decode_state_bytes", "llattn_decode_step",
+    "llattn_bwd_workspace_bytes", "llattn_bwd",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20  # LLATTN_NOALLOC_SCRATCH_BYTES
@@ -74,6 +75,11 @@ def lib():
     L.llattn_decode_state_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
     L.llattn_decode_step.restype = i
     L.llattn_decode_step.argtypes = [i, vp, vp, vp, f_p, f_p, i_p, f_p, f_p, i, i, i, i, i, vp]
+    L.llattn_bwd_workspace_bytes.restype = i
+    L.llattn_bwd_workspace_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+    L.llattn_bwd.restype = i
+    L.llattn_bwd.argtypes = [i, vp, vp, vp, f_p, f_p, vp, f_p, f_p, f_p, f_p, f_p, i, i, i, i, i,
+                             i_p, vp, ctypes.c_size_t, vp]
     L.llattn_profile.restype = i
     L.llattn_profile.argtypes = [i]
     L.llattn_profile_read.restype = i
@@ -232,6 +238,50 @@ def decode_step(q, k, v, log_a, lam, pos, state, out, B, H, L, dk, dv, stream=No
                                   int(dk), int(dv), _stream_handle(stream))
     _check(st, "llattn_decode_step")
     return out
+
+
+def bwd_workspace_bytes(B: int, H: int, T: int, dk: int, dv: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().llattn_bwd_workspace_bytes(int(B), int(H), int(T), int(dk), int(dv),
+                                            ctypes.byref(n)), "llattn_bwd_workspace_bytes")
+    return int(n.value)
+
+
+def backward(q, k, v, log_a, lam, dout, *, cu_seqlens=None, T: Optional[int] = None,
+             grads=None, workspace=None, stream=None):
+    """Gradients of sum(dout * out) through llattn_bwd, on device tensors (torch).
+
+    Shapes as in forward(); dout like out, in the dtype of q.  Returns a dict of fp32 tensors
+    q, k, v, log_a, lam (or fills `grads`, a dict of preallocated ones)."""
+    import torch
+    in_dtype = BF16 if q.dtype == torch.bfloat16 else F32
+    for t in (q, k, v, log_a, lam, dout):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if k.dtype != q.dtype or v.dtype != q.dtype or dout.dtype != q.dtype:
+        raise TypeError("q, k, v and dout must share a dtype")
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape
+    else:
+        B = cu_seqlens.numel() - 1
+        _, H, dk = q.shape
+        if T is None:
+            raise ValueError("varlen needs T (max sequence length bound)")
+    dv = v.shape[-1]
+    if grads is None:
+        grads = {n: torch.empty(x.shape, dtype=torch.float32, device=x.device)
+                 for n, x in (("q", q), ("k", k), ("v", v), ("log_a", log_a), ("lam", lam))}
+    ws_ptr, ws_n = None, 0
+    if workspace is not None:
+        ws_ptr, ws_n = ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = lib().llattn_bwd(in_dtype, P(q), P(k), P(v), P(log_a), P(lam), P(dout), P(grads["q"]),
+                          P(grads["k"]), P(grads["v"]), P(grads["log_a"]), P(grads["lam"]),
+                          int(B), int(H), int(T), int(dk), int(dv),
+                          P(cu_seqlens) if cu_seqlens is not None else None, ws_ptr, ws_n,
+                          _stream_handle(stream))
+    _check(st, "llattn_bwd")
+    return grads
 
 
 def profile(enable: bool):

@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "../../include/llattn.h"
+#include "llattn_bwd.h"
 #include "llattn_decode.h"
 #include "llattn_internal.h"
 
@@ -96,6 +97,34 @@ llattn_status device_state(DeviceState** out, int* dev_out) {
   return LLATTN_OK;
 }
 
+// The scratch of one call: the caller's workspace (checked for size and alignment), or the
+// library's per-device buffer, grown on demand under `lock`, which stays held for the launch.
+llattn_status pick_workspace(DeviceState* ds, size_t need, void* workspace, size_t workspace_bytes,
+                             std::unique_lock<std::mutex>& lock, void** ws) {
+  *ws = workspace;
+  if (workspace != nullptr) {
+    if (workspace_bytes < need || !aligned(workspace, 256)) return LLATTN_ERR_WORKSPACE;
+  } else if (need > 0) {
+    lock.lock();
+    if (ds->ws_bytes < need) {
+      cudaError_t e;
+      if (ds->ws) {
+        if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
+        cudaFree(ds->ws);
+        ds->ws = nullptr;
+        ds->ws_bytes = 0;
+      }
+      if ((e = cudaMalloc(&ds->ws, need)) != cudaSuccess) {
+        ds->ws = nullptr;
+        return cuda_fail(e);
+      }
+      ds->ws_bytes = need;
+    }
+    *ws = ds->ws;
+  }
+  return LLATTN_OK;
+}
+
 llattn_status forward(int in_dtype, int path, int chunk, const void* q, const void* k,
                       const void* v, const float* log_a, const float* lam, float* out, int B,
                       int H, int T, int dk, int dv, const int* cu_seqlens, void* workspace,
@@ -135,26 +164,7 @@ llattn_status forward(int in_dtype, int path, int chunk, const void* q, const vo
   const size_t need = workspace_for(path, chunk, B, H, T, dk, dv);
   void* ws = workspace;
   std::unique_lock<std::mutex> lock(g_mu, std::defer_lock);
-  if (workspace != nullptr) {
-    if (workspace_bytes < need || !aligned(workspace, 256)) return LLATTN_ERR_WORKSPACE;
-  } else if (need > 0) {
-    lock.lock();
-    if (ds->ws_bytes < need) {
-      cudaError_t e;
-      if (ds->ws) {
-        if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
-        cudaFree(ds->ws);
-        ds->ws = nullptr;
-        ds->ws_bytes = 0;
-      }
-      if ((e = cudaMalloc(&ds->ws, need)) != cudaSuccess) {
-        ds->ws = nullptr;
-        return cuda_fail(e);
-      }
-      ds->ws_bytes = need;
-    }
-    ws = ds->ws;
-  }
+  if ((s = pick_workspace(ds, need, workspace, workspace_bytes, lock, &ws)) != LLATTN_OK) return s;
   llattn::Problem p{in_dtype, q, k, v, log_a, lam, out, B, H, T, dk, dv, L, cu_seqlens,
                     ds->status};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -522,6 +532,63 @@ llattn_status llattn_decode_step(int in_dtype, const void* q, const void* k, con
   llattn::DecodeProblem p{in_dtype, q, k, v, log_a, lam, pos, state, state + nlev, out,
                           B, H, L, dk, dv, ds->status};
   const cudaError_t e = llattn::decode_step(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_bwd_workspace_bytes(int B, int H, int T, int dk, int dv, size_t* bytes) {
+  if (!bytes) return LLATTN_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || T > (1 << 24) || H > 65535 || B > 65535) return LLATTN_ERR_SHAPE;
+  if (dk != dv || (dk != 32 && dk != 64)) return LLATTN_ERR_SHAPE;
+  *bytes = (B == 0 || H == 0 || T == 0) ? 0 : llattn::bwd_workspace_bytes(B, H, T);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_bwd(int in_dtype, const void* q, const void* k, const void* v,
+                         const float* log_a, const float* lam, const void* dout, float* dq,
+                         float* dk, float* dv, float* dlog_a, float* dlam, int B, int H, int T,
+                         int dk_dim, int dv_dim, const int* cu_seqlens, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+  size_t need = 0;
+  llattn_status s = llattn_bwd_workspace_bytes(B, H, T, dk_dim, dv_dim, &need);
+  if (s != LLATTN_OK) return s;
+  if (B == 0 || H == 0 || T == 0) return LLATTN_OK;  // nothing to compute
+  const void* ptrs[12] = {q, k, v, log_a, lam, dout, dq, dk, dv, dlog_a, dlam, nullptr};
+  for (int i = 0; i < 11; ++i)
+    if (ptrs[i] == nullptr) return LLATTN_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(log_a, 4) ||
+      !aligned(lam, 4) || !aligned(dlog_a, 4) || !aligned(dlam, 4) ||
+      (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return LLATTN_ERR_ALIGN;
+  const int L = llattn_num_levels(T);
+  if (cu_seqlens == nullptr) {
+    // dense: no gradient may overlap an input or another gradient
+    const size_t ntok = (size_t)B * T * H, d = (size_t)dk_dim;
+    const size_t esz = in_dtype == LLATTN_BF16 ? 2 : 4;
+    const struct { const void* p; size_t n; } rng[11] = {
+        {q, ntok * d * esz}, {k, ntok * d * esz}, {v, ntok * d * esz}, {dout, ntok * d * esz},
+        {log_a, ntok * 4}, {lam, ntok * L * 4}, {dq, ntok * d * 4}, {dk, ntok * d * 4},
+        {dv, ntok * d * 4}, {dlog_a, ntok * 4}, {dlam, ntok * L * 4}};
+    for (int o = 6; o < 11; ++o) {
+      const uintptr_t o0 = reinterpret_cast<uintptr_t>(rng[o].p), o1 = o0 + rng[o].n;
+      for (int i = 0; i < 11; ++i) {
+        if (i == o) continue;
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(rng[i].p), a1 = a0 + rng[i].n;
+        if (a0 < o1 && o0 < a1) return LLATTN_ERR_ARG;
+      }
+    }
+  }
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  if ((s = device_state(&ds, &dev)) != LLATTN_OK) return s;
+  void* ws = nullptr;
+  std::unique_lock<std::mutex> lock(g_mu, std::defer_lock);
+  if ((s = pick_workspace(ds, need, workspace, workspace_bytes, lock, &ws)) != LLATTN_OK) return s;
+  llattn::BwdProblem p{in_dtype, q, k, v, dout, log_a, lam, dq, dk, dv, dlog_a, dlam,
+                       B, H, T, dk_dim, L, cu_seqlens, ds->status};
+  const cudaError_t e = llattn::bwd(p, ws, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return LLATTN_OK;
 }

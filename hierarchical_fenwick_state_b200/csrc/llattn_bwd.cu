@@ -1,0 +1,361 @@
+// Backward pass of log-linear attention (Mamba-2 form): the gradients of sum(dout * out) with
+// respect to q, k, v, log_a and lam.
+//
+// Log-Linear Attention (gist.science summaries, Italian "Sommario tecnico" section 2, "Matrici
+// Gerarchiche"): the output is ((Q K^T) .* M_H) V with M_H a hierarchical (HODLR) mask.  Read
+// level by level, M_H has a simple block form: at level l >= 1 the positions fall into aligned
+// blocks of 2^l tokens, and every key s in a block's left half meets every query t in its right
+// half at level l, with weight lam[t, l] * exp(g_t - g_s) (g the inclusive prefix sum of log_a).
+// With m the last position of the left half, exp(g_t - g_s) = exp(g_t - g_m) * exp(g_m - g_s),
+// so each block's interaction has rank d and the backward needs, per block, only
+//
+//   S = sum over left-half s of exp(g_m - g_s) k_s v_s^T          (d x d)
+//   U = sum over right-half t of lam[t,l] exp(g_t - g_m) q_t do_t^T (d x d)
+//
+// from which, for t in the right half and s in the left half,
+//
+//   w_t = exp(g_t - g_m) S do_t,    dlam[t, l] = q_t . w_t,    dq_t += lam[t, l] w_t,
+//   dk_s += exp(g_m - g_s) U v_s,   dv_s += exp(g_m - g_s) U^T k_s,
+//
+// and dlam[s, l] = 0 on the left half (a left-half token has no partner at that level).
+// Levels 0..5 (pairs inside an aligned 32-token tile) are done densely per tile: the score and
+// gradient-score tiles, the mask, and the three small products.  The gate gradient follows from
+// the row and column sums of the exponent's gradient, which equal q_t . dq_t and k_t . dk_t:
+// dg_t = q_t . dq_t - k_t . dk_t, and dlog_a[r] = sum over t >= r of dg_t.
+//
+// Kernels, in stream order: the prefix sums g (fp64: the differences of long prefix sums must
+// stay exact), the dense tiles (they initialise dq, dk, dv and dlam[:, 0..5]), one launch per
+// level 6..L-1 (each token sits in one block per level, so the updates of one launch never
+// collide), and the reverse scan for dlog_a.  Arithmetic is fp32 on CUDA cores; d = dk = dv in
+// {32, 64}.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/llattn.h"
+#include "llattn_bwd.h"
+#include "llattn_common.cuh"
+#include "llattn_internal.h"
+
+namespace llattn {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kTile = 32;        // dense tile: levels 0..5
+constexpr int kDenseLevels = 6;
+constexpr int kThreads = 256;
+
+// ---- g: inclusive prefix sums of log_a per (sequence, head), one warp each ----
+__global__ void bwd_prefix_g(BwdProblem p, double* g) {
+  const int h = blockIdx.x, sq = blockIdx.y, lane = threadIdx.x;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  double carry = 0.0;
+  for (int base = 0; base < sp.len; base += 32) {
+    const int t = base + lane;
+    const size_t row = (size_t)(sp.start + t) * p.H + h;
+    double x = t < sp.len ? (double)p.log_a[row] : 0.0;   // row is read only for t < len
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double y = __shfl_up_sync(kFull, x, off);
+      if (lane >= off) x += y;
+    }
+    x += carry;
+    if (t < sp.len) g[((size_t)sq * p.T + t) * p.H + h] = x;
+    carry = __shfl_sync(kFull, x, 31);
+  }
+}
+
+// ---- levels 0..5: dense 32 x 32 tiles ----
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kThreads) bwd_dense_tile(BwdProblem p, const double* g) {
+  __shared__ float s_q[kTile][D + 1], s_k[kTile][D + 1], s_v[kTile][D + 1], s_do[kTile][D + 1];
+  __shared__ float s_pm[kTile][kTile + 1];  // (do_i . v_j) M[i, j]
+  __shared__ float s_pa[kTile][kTile + 1];  // (q_i . k_j) M[i, j]
+  __shared__ float s_x[kTile][kTile + 1];   // (do_i . v_j)(q_i . k_j) exp(g_i - g_j)
+  __shared__ double s_g[kTile];
+  __shared__ float s_lam[kTile][kDenseLevels];
+
+  const int tile = blockIdx.x, h = blockIdx.y, sq = blockIdx.z, tid = threadIdx.x;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  const int t0 = tile * kTile;
+  if (t0 >= sp.len) return;
+  const int n = min(kTile, sp.len - t0);
+  const Tin* q = static_cast<const Tin*>(p.q);
+  const Tin* k = static_cast<const Tin*>(p.k);
+  const Tin* v = static_cast<const Tin*>(p.v);
+  const Tin* dout = static_cast<const Tin*>(p.dout);
+  const size_t row0 = (size_t)(sp.start + t0) * p.H + h;  // row of token t0; next token + H
+
+  for (int e = tid; e < kTile * D; e += kThreads) {
+    const int i = e / D, c = e % D;
+    const bool ok = i < n;
+    const size_t off = (row0 + (size_t)i * p.H) * D + c;
+    s_q[i][c] = ok ? ld_in(q + off) : 0.f;
+    s_k[i][c] = ok ? ld_in(k + off) : 0.f;
+    s_v[i][c] = ok ? ld_in(v + off) : 0.f;
+    s_do[i][c] = ok ? ld_in(dout + off) : 0.f;
+  }
+  const size_t grow0 = ((size_t)sq * p.T + t0) * p.H + h;  // g is indexed by local position
+  if (tid < kTile) s_g[tid] = tid < n ? g[grow0 + (size_t)tid * p.H] : 0.0;
+  for (int e = tid; e < kTile * kDenseLevels; e += kThreads) {
+    const int i = e / kDenseLevels, l = e % kDenseLevels;
+    s_lam[i][l] = (i < n && l < p.L) ? p.lam[(row0 + (size_t)i * p.H) * p.L + l] : 0.f;
+  }
+  __syncthreads();
+
+  // pair tiles; positions t0+i, t0+j share the tile, so their level is that of (i, j)
+  for (int e = tid; e < kTile * kTile; e += kThreads) {
+    const int i = e / kTile, j = e % kTile;
+    float pm = 0.f, pa = 0.f, x = 0.f;
+    if (j <= i && i < n) {
+      float a = 0.f, b = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) {
+        a = fmaf(s_q[i][c], s_k[j][c], a);
+        b = fmaf(s_do[i][c], s_v[j][c], b);
+      }
+      const float E = expf((float)(s_g[i] - s_g[j]));
+      const float m = s_lam[i][fenwick_level(i, j)] * E;
+      pm = b * m;
+      pa = a * m;
+      x = a * b * E;
+    }
+    s_pm[i][j] = pm;
+    s_pa[i][j] = pa;
+    s_x[i][j] = x;
+  }
+  __syncthreads();
+
+  // dlam[:, 0..5]: sums of s_x over each level's keys
+  if (tid < kTile * kDenseLevels) {
+    const int i = tid / kDenseLevels, l = tid % kDenseLevels;
+    if (i < n && l < p.L) {
+      float s = 0.f;
+      for (int j = 0; j <= i; ++j)
+        if (fenwick_level(i, j) == l) s += s_x[i][j];
+      p.dlam[(row0 + (size_t)i * p.H) * p.L + l] = s;
+    }
+  }
+  // dq = Pm K, dk = Pm^T Q, dv = Pa^T dO  (they start the accumulation of the later levels)
+  for (int e = tid; e < kTile * D; e += kThreads) {
+    const int i = e / D, c = e % D;
+    if (i >= n) continue;
+    float aq = 0.f, ak = 0.f, av = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < kTile; ++j) {
+      aq = fmaf(s_pm[i][j], s_k[j][c], aq);
+      ak = fmaf(s_pm[j][i], s_q[j][c], ak);
+      av = fmaf(s_pa[j][i], s_do[j][c], av);
+    }
+    const size_t off = (row0 + (size_t)i * p.H) * D + c;
+    p.dq[off] = aq;
+    p.dk[off] = ak;
+    p.dv[off] = av;
+  }
+}
+
+// ---- one level >= 6: the rank-d interaction of each aligned block's halves ----
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kThreads) bwd_level_block(BwdProblem p, const double* g, int lvl) {
+  constexpr int R = D * D / kThreads;  // state elements per thread
+  constexpr int W = D / 32;            // outputs per lane in the per-token products
+  __shared__ float s_mem[2 * D * (D + 1)];  // phase 1: staged rows; phase 2: S and U
+  __shared__ float s_w[32];
+  float (*s_x)[D] = reinterpret_cast<float (*)[D]>(s_mem);               // [32][D]
+  float (*s_y)[D] = reinterpret_cast<float (*)[D]>(s_mem + 32 * D);      // [32][D]
+  float (*s_S)[D + 1] = reinterpret_cast<float (*)[D + 1]>(s_mem);       // [D][D+1]
+  float (*s_U)[D + 1] = reinterpret_cast<float (*)[D + 1]>(s_mem + D * (D + 1));
+
+  const int blk = blockIdx.x, h = blockIdx.y, sq = blockIdx.z, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  const int half = 1 << (lvl - 1);
+  const long long a0 = (long long)blk << lvl;
+  if (a0 >= sp.len) return;
+  const int lo = (int)a0;
+  const int mid = lo + half;                           // first token of the right half
+  const int lend = min(mid, sp.len);                   // left half [lo, lend)
+  const int rend = (int)min((long long)lo + 2 * half, (long long)sp.len);  // right [mid, rend)
+  const Tin* q = static_cast<const Tin*>(p.q);
+  const Tin* k = static_cast<const Tin*>(p.k);
+  const Tin* v = static_cast<const Tin*>(p.v);
+  const Tin* dout = static_cast<const Tin*>(p.dout);
+  auto row = [&](int t) { return (size_t)(sp.start + t) * p.H + h; };
+  auto grow = [&](int t) { return ((size_t)sq * p.T + t) * p.H + h; };
+
+  for (int t = lo + tid; t < lend; t += kThreads) p.dlam[row(t) * p.L + lvl] = 0.f;
+  if (mid >= sp.len) return;  // no right half: nothing meets at this level
+  const double gm = g[grow(mid - 1)];
+
+  // phase 1: S over the left half, U over the right half
+  float accS[R], accU[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) accS[r] = accU[r] = 0.f;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int b0 = pass == 0 ? lo : mid, b1 = pass == 0 ? lend : rend;
+    for (int base = b0; base < b1; base += 32) {
+      if (tid < 32) {
+        const int t = base + tid;
+        float w = 0.f;
+        if (t < b1)
+          w = pass == 0 ? expf((float)(gm - g[grow(t)]))
+                        : p.lam[row(t) * p.L + lvl] * expf((float)(g[grow(t)] - gm));
+        s_w[tid] = w;
+      }
+      __syncthreads();
+      for (int e = tid; e < 32 * D; e += kThreads) {
+        const int i = e / D, c = e % D;
+        const int t = base + i;
+        float x = 0.f, y = 0.f;
+        if (t < b1) {
+          const size_t off = row(t) * D + c;
+          x = s_w[i] * (pass == 0 ? ld_in(k + off) : ld_in(q + off));
+          y = pass == 0 ? ld_in(v + off) : ld_in(dout + off);
+        }
+        s_x[i][c] = x;
+        s_y[i][c] = y;
+      }
+      __syncthreads();
+      const int nrow = min(32, b1 - base);
+      for (int i = 0; i < nrow; ++i) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int e = tid + r * kThreads, a = e / D, b = e % D;
+          if (pass == 0) accS[r] = fmaf(s_x[i][a], s_y[i][b], accS[r]);
+          else accU[r] = fmaf(s_x[i][a], s_y[i][b], accU[r]);
+        }
+      }
+      __syncthreads();
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = tid + r * kThreads, a = e / D, b = e % D;
+    s_S[a][b] = accS[r];
+    s_U[a][b] = accU[r];
+  }
+  __syncthreads();
+
+  // phase 2, right half (one warp per token): w = e^{g_t - g_m} S do_t; dlam; dq
+  for (int t = mid + warp; t < rend; t += kThreads / 32) {
+    const size_t rr = row(t);
+    float dol[W], ql[W], wl[W];
+#pragma unroll
+    for (int u = 0; u < W; ++u) {
+      dol[u] = ld_in(dout + rr * D + lane + 32 * u);
+      ql[u] = ld_in(q + rr * D + lane + 32 * u);
+      wl[u] = 0.f;
+    }
+#pragma unroll
+    for (int u2 = 0; u2 < W; ++u2)
+      for (int bb = 0; bb < 32; ++bb) {
+        const float dob = __shfl_sync(kFull, dol[u2], bb);
+        const int b = bb + 32 * u2;
+#pragma unroll
+        for (int u = 0; u < W; ++u) wl[u] = fmaf(s_S[lane + 32 * u][b], dob, wl[u]);
+      }
+    const float sc = expf((float)(g[grow(t)] - gm));
+    const float lam = p.lam[rr * p.L + lvl];
+    float dl = 0.f;
+#pragma unroll
+    for (int u = 0; u < W; ++u) {
+      wl[u] *= sc;
+      dl = fmaf(ql[u], wl[u], dl);
+      p.dq[rr * D + lane + 32 * u] += lam * wl[u];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dl += __shfl_xor_sync(kFull, dl, off);
+    if (lane == 0) p.dlam[rr * p.L + lvl] = dl;
+  }
+
+  // phase 2, left half: dk_s += e^{g_m - g_s} U v_s, dv_s += e^{g_m - g_s} U^T k_s
+  for (int s = lo + warp; s < lend; s += kThreads / 32) {
+    const size_t rr = row(s);
+    float vl[W], kl[W], ak[W], av[W];
+#pragma unroll
+    for (int u = 0; u < W; ++u) {
+      vl[u] = ld_in(v + rr * D + lane + 32 * u);
+      kl[u] = ld_in(k + rr * D + lane + 32 * u);
+      ak[u] = av[u] = 0.f;
+    }
+#pragma unroll
+    for (int u2 = 0; u2 < W; ++u2)
+      for (int bb = 0; bb < 32; ++bb) {
+        const int b = bb + 32 * u2;
+        const float vb = __shfl_sync(kFull, vl[u2], bb);
+        const float kb = __shfl_sync(kFull, kl[u2], bb);
+#pragma unroll
+        for (int u = 0; u < W; ++u) {
+          ak[u] = fmaf(s_U[lane + 32 * u][b], vb, ak[u]);   // (U v)[a],   a = lane + 32u
+          av[u] = fmaf(s_U[b][lane + 32 * u], kb, av[u]);   // (U^T k)[c], c = lane + 32u
+        }
+      }
+    const float sc = expf((float)(gm - g[grow(s)]));
+#pragma unroll
+    for (int u = 0; u < W; ++u) {
+      p.dk[rr * D + lane + 32 * u] += sc * ak[u];
+      p.dv[rr * D + lane + 32 * u] += sc * av[u];
+    }
+  }
+}
+
+// ---- dlog_a: reverse prefix sums of dg_t = q_t . dq_t - k_t . dk_t, one warp each ----
+template <typename Tin, int D>
+__global__ void bwd_dlog_a(BwdProblem p) {
+  const int h = blockIdx.x, sq = blockIdx.y, lane = threadIdx.x;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  const Tin* q = static_cast<const Tin*>(p.q);
+  const Tin* k = static_cast<const Tin*>(p.k);
+  double carry = 0.0;
+  for (int end = sp.len; end > 0; end -= 32) {
+    const int t = end - 32 + lane;
+    double x = 0.0;
+    if (t >= 0) {
+      const size_t rr = (size_t)(sp.start + t) * p.H + h;
+      float a = 0.f;
+      for (int c = 0; c < D; ++c)
+        a += ld_in(q + rr * D + c) * p.dq[rr * D + c] - ld_in(k + rr * D + c) * p.dk[rr * D + c];
+      x = a;
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double y = __shfl_down_sync(kFull, x, off);
+      if (lane + off < 32) x += y;
+    }
+    x += carry;
+    if (t >= 0) p.dlog_a[(size_t)(sp.start + t) * p.H + h] = (float)x;
+    carry = __shfl_sync(kFull, x, 0);
+  }
+}
+
+template <typename Tin, int D>
+cudaError_t launch(const BwdProblem& p, double* g, cudaStream_t st) {
+  const dim3 seqs(p.H, p.nseq);
+  bwd_prefix_g<<<seqs, 32, 0, st>>>(p, g);
+  bwd_dense_tile<Tin, D><<<dim3((p.T + kTile - 1) / kTile, p.H, p.nseq), kThreads, 0, st>>>(p, g);
+  int n = 2;
+  for (int lvl = kDenseLevels; lvl < p.L; ++lvl, ++n) {
+    const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
+    bwd_level_block<Tin, D><<<dim3(nblk, p.H, p.nseq), kThreads, 0, st>>>(p, g, lvl);
+  }
+  bwd_dlog_a<Tin, D><<<seqs, 32, 0, st>>>(p);
+  count_launch(n + 1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t bwd(const BwdProblem& p, void* ws, cudaStream_t st) {
+  double* g = static_cast<double*>(ws);
+  main_kernel_begin(st);
+  cudaError_t e;
+  if (p.in_dtype == LLATTN_BF16)
+    e = p.d == 32 ? launch<__nv_bfloat16, 32>(p, g, st) : launch<__nv_bfloat16, 64>(p, g, st);
+  else
+    e = p.d == 32 ? launch<float, 32>(p, g, st) : launch<float, 64>(p, g, st);
+  main_kernel_end(st);
+  return e;
+}
+
+}  // namespace llattn

@@ -276,6 +276,46 @@ LLATTN_API llattn_status llattn_decode_step(int in_dtype, const void* q, const v
                                             int H, int L, int dk, int dv, void* stream);
 
 /*
+ * Backward pass: the gradients of sum(dout * out) with respect to q, k, v, log_a and lam, for
+ * the operation llattn_fwd computes (same inputs, same layouts, dense or packed).
+ *
+ * Log-Linear Attention (gist.science summaries, Italian "Sommario tecnico" section 2, "Matrici
+ * Gerarchiche"): out = ((Q K^T) .* M_H) V with M_H the hierarchical (HODLR) mask
+ * M_H[t, s] = lam[t, l(t, s)] * prod_{r=s+1..t} a_r.  Level by level, the mask couples the
+ * left and right halves of aligned blocks of 2^l positions with a rank-d factor, and the
+ * gradients are computed that way:
+ *   dq_t   = sum_{s<=t} M_H[t,s] (dout_t . v_s) k_s      dk_s = sum_{t>=s} M_H[t,s] (dout_t . v_s) q_t
+ *   dv_s   = sum_{t>=s} M_H[t,s] (q_t . k_s) dout_t
+ *   dlam[t, l]  = sum over s with l(t,s) == l of prod a * (q_t . k_s)(dout_t . v_s)
+ *   dlog_a[r]   = sum over t >= r of (q_t . dq_t - k_t . dk_t)   (positions within a sequence)
+ * dlam is zero at levels a token has no partner at; dlog_a at a sequence's first position is
+ * zero up to rounding (no gate product contains it).
+ *
+ * llattn_bwd_workspace_bytes - scratch llattn_bwd needs: B*T*H*8 bytes (fp64 prefix sums of
+ * log_a), rounded up to 256.  dk == dv in {32, 64}; other head sizes return LLATTN_ERR_SHAPE.
+ *
+ * llattn_bwd
+ *   in_dtype   LLATTN_BF16 or LLATTN_F32: the type of q, k, v and dout (bf16 as uint16 bit
+ *              patterns).  Arithmetic is fp32 on CUDA cores.
+ *   q, k, v, log_a, lam, B, H, T, cu_seqlens   as in llattn_fwd.
+ *   dout       [B, T, H, dv] (packed: [total, H, dv]), the gradient of the loss at out.
+ *   dq, dk, dv [.., H, d] fp32; dlog_a [.., H] fp32; dlam [.., H, L] fp32: fully overwritten
+ *              for every token of every sequence.
+ *   workspace  caller-owned device scratch of llattn_bwd_workspace_bytes() bytes (256-byte
+ *              aligned), or NULL for the library's per-device buffer (as llattn_fwd).
+ * Pointers: q, k, v, dout, dq, dk, dv 16-byte aligned, the rest 4-byte aligned; no gradient
+ * may overlap an input or another gradient.  Asynchronous on `stream`.
+ */
+LLATTN_API llattn_status llattn_bwd_workspace_bytes(int B, int H, int T, int dk, int dv,
+                                                    size_t* bytes);
+LLATTN_API llattn_status llattn_bwd(int in_dtype, const void* q, const void* k, const void* v,
+                                    const float* log_a, const float* lam, const void* dout,
+                                    float* dq, float* dk, float* dv, float* dlog_a, float* dlam,
+                                    int B, int H, int T, int dk_dim, int dv_dim,
+                                    const int* cu_seqlens, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
  * Launch accounting, for benchmarks.  llattn_profile(1) starts recording a pair
  * of CUDA events on the call's stream around the dominant kernel of every
  * forward (the one that streams q, k, v, lam and writes out); llattn_profile(0)

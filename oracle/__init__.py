@@ -9,5 +9,5 @@ from .llattn_oracle import (  # noqa: F401
     llattn_single, llattn_bruteforce, llattn_quadratic, llattn_recurrent, mamba2_recurrent,
     llattn_sampled, rel_max_err,
     llattn_level_states, llattn_decode_step, llattn_decode_sequence, llattn_decode_batch,
-    llattn_backward_seq, llattn_backward,
+    llattn_backward_seq, llattn_backward, llattn_backward_sampled,
 )

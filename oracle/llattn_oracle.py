@@ -472,3 +472,48 @@ def llattn_backward(inp, do):
     return {"q": res["q"].reshape(inp.q.shape), "k": res["k"].reshape(inp.k.shape),
             "v": res["v"].reshape(inp.v.shape), "log_a": res["log_a"].reshape(inp.log_a.shape),
             "lam": res["lam"].reshape(inp.lam.shape)}
+
+
+def llattn_backward_sampled(inp, do, samples):
+    """Gradient rows at sampled (token_index, head) pairs of the flattened [tokens, H] grid,
+    each by direct summation over its own row or column of the mask (the definition):
+      dq_t  = sum_{s<=t} M[t,s] (do_t . v_s) k_s,     dlam[t, l] = sum_{l(t,s)=l} E[t,s] (q_t . k_s)(do_t . v_s),
+      dk_s  = sum_{t>=s} M[t,s] (do_t . v_s) q_t,     dv_s = sum_{t>=s} M[t,s] (q_t . k_s) do_t,
+    with E[t, s] the gate product as exp of a sum of log_a and M[t, s] = lam[t, l(t,s)] E[t, s].
+    Returns dict q, k, v [n, d] and lam [n, L] (fp64)."""
+    qf = np.asarray(inp.q, F64).reshape(-1, inp.H, inp.dk)
+    kf = np.asarray(inp.k, F64).reshape(-1, inp.H, inp.dk)
+    vf = np.asarray(inp.v, F64).reshape(-1, inp.H, inp.dv)
+    laf = np.asarray(inp.log_a, F64).reshape(-1, inp.H)
+    lmf = np.asarray(inp.lam, F64).reshape(-1, inp.H, inp.L)
+    dof = np.asarray(do, F64).reshape(-1, inp.H, inp.dv)
+    starts = np.array([s for s, _ in inp.seq_slices()], np.int64)
+    lens = np.array([n for _, n in inp.seq_slices()], np.int64)
+    n = len(samples)
+    out = {"q": np.zeros((n, inp.dk)), "k": np.zeros((n, inp.dk)), "v": np.zeros((n, inp.dv)),
+           "lam": np.zeros((n, inp.L))}
+    for i, (tok, h) in enumerate(samples):
+        sq = int(np.searchsorted(starts, tok, side="right") - 1)
+        s0, ln = int(starts[sq]), int(lens[sq])
+        x = tok - s0                                   # sequence-local position
+        la = laf[s0:s0 + ln, h]
+        # row x: keys s <= x; gate product over r = s+1..x
+        ks = np.arange(x + 1)
+        pref = np.concatenate([[0.0], np.cumsum(la[1:x + 1])])     # sum of la[1..j]
+        E_row = np.exp(pref[x] - pref[ks])
+        lev_row = fenwick_level_matrix(np.array([x]), ks)[0]
+        a_row = kf[s0 + ks, h] @ qf[tok, h]
+        b_row = vf[s0 + ks, h] @ dof[tok, h]
+        m_row = lmf[tok, h][lev_row] * E_row
+        out["q"][i] = (m_row * b_row) @ kf[s0 + ks, h]
+        np.add.at(out["lam"][i], lev_row, E_row * a_row * b_row)
+        # column x: queries t >= x; gate product over r = x+1..t
+        ts = np.arange(x, ln)
+        E_col = np.exp(np.cumsum(np.concatenate([[0.0], la[x + 1:ln]])))
+        lev_col = fenwick_level_matrix(ts, np.array([x]))[:, 0]
+        m_col = lmf[s0 + ts, h][np.arange(len(ts)), lev_col] * E_col
+        a_col = qf[s0 + ts, h] @ kf[tok, h]
+        b_col = dof[s0 + ts, h] @ vf[tok, h]
+        out["k"][i] = (m_col * b_col) @ qf[s0 + ts, h]
+        out["v"][i] = (m_col * a_col) @ dof[s0 + ts, h]
+    return out

@@ -138,3 +138,43 @@ def test_decode_argument_errors_before_launch(kw, status):
 def test_decode_empty_batches_are_no_ops():
     assert _decode(B=0) == 0
     assert _decode(H=0) == 0
+
+
+def _bwd(**kw):
+    a = dict(in_dtype=1, q=0x1000, k=0x2000, v=0x3000, log_a=0x4000, lam=0x5000, dout=0x6000,
+             dq=0x10000, dk=0x20000, dv=0x30000, dlog_a=0x40000, dlam=0x50000, B=1, H=2, T=16,
+             dk_dim=64, dv_dim=64, cu=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return binding.lib().llattn_bwd(a["in_dtype"], vp(a["q"]), vp(a["k"]), vp(a["v"]),
+                                    vp(a["log_a"]), vp(a["lam"]), vp(a["dout"]), vp(a["dq"]),
+                                    vp(a["dk"]), vp(a["dv"]), vp(a["dlog_a"]), vp(a["dlam"]),
+                                    a["B"], a["H"], a["T"], a["dk_dim"], a["dv_dim"],
+                                    vp(a["cu"]) if a["cu"] else None, None, 0, None)
+
+
+def test_bwd_workspace_bytes():
+    assert binding.bwd_workspace_bytes(4, 32, 8192, 64, 64) == 4 * 32 * 8192 * 8
+    assert binding.bwd_workspace_bytes(1, 3, 5, 32, 32) == 256          # rounded up to 256
+    assert binding.bwd_workspace_bytes(0, 3, 5, 32, 32) == 0
+    for bad in ((1, 1, 16, 64, 32), (1, 1, 16, 128, 128), (1, 1, -1, 64, 64)):
+        with pytest.raises(binding.LLAttnError) as e:
+            binding.bwd_workspace_bytes(*bad)
+        assert e.value.status == 2
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk_dim=32), 2), (dict(dk_dim=128, dv_dim=128), 2), (dict(T=-1), 2),
+    (dict(in_dtype=3), 4),
+    (dict(dout=0), 1), (dict(dlam=0), 1),
+    (dict(dq=0x10008), 3), (dict(dout=0x6008), 3), (dict(dlog_a=0x40002), 3),
+    # a gradient overlapping an input (dout: 16 tokens x 2 heads x 64 x 2 B from 0x6000) or
+    # another gradient (dq: 16 x 2 x 64 x 4 B = 8 KB from 0x10000)
+    (dict(dq=0x6100), 1), (dict(dk=0x10400), 1),
+])
+def test_bwd_argument_errors_before_launch(kw, status):
+    assert _bwd(**kw) == status
+
+
+def test_bwd_empty_problems_are_no_ops():
+    assert _bwd(B=0) == 0 and _bwd(H=0) == 0 and _bwd(T=0) == 0

@@ -1,0 +1,108 @@
+"""Backward pass on the GPU (llattn_bwd through the C ABI) against the oracle.
+
+Every gradient (dq, dk, dv, dlog_a, dlam) is compared element by element with the
+oracle's backward at sizes it finishes in seconds: several levels of blocks and a
+ragged tail, one token, a packed batch with an empty and a one-token sequence, bf16
+and fp32 inputs, slow and the workloads' own decay.  At the benchmark's size (B=4,
+H=32, T=8192, d=64) sampled gradient rows and columns are compared with the oracle's
+direct sums.  The kernels compute in fp32 on the exact input values, so the bound is
+1e-4 of each gradient's RMS for bf16 inputs too.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from hierarchical_fenwick_state_b200 import binding
+from hierarchical_fenwick_state_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-4
+W = I.WORKLOADS
+NAMES = ("q", "k", "v", "log_a", "lam")
+
+
+def _run(inp, do):
+    import torch
+    tdt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    dev = torch.device("cuda:0")
+    t = {n: torch.from_numpy(getattr(inp, n)).to(dev) for n in NAMES}
+    for n in ("q", "k", "v"):
+        t[n] = t[n].to(tdt)
+    tdo = torch.from_numpy(do.astype(np.float32)).to(dev).to(tdt)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev) if inp.cu_seqlens is not None else None
+    grads = {n: torch.full(getattr(inp, n).shape, float("nan"), dtype=torch.float32, device=dev)
+             for n in NAMES}
+    binding.device_status(clear=True)
+    binding.backward(t["q"], t["k"], t["v"], t["log_a"], t["lam"], tdo, cu_seqlens=cu, T=inp.T,
+                     grads=grads)
+    torch.cuda.synchronize()
+    assert binding.device_status(clear=True) == 0
+    return {n: g.double().cpu().numpy() for n, g in grads.items()}
+
+
+def _check(got, ref):
+    """Each gradient within TOL of its RMS.  A gradient that is zero in exact arithmetic (dlog_a
+    of one-token sequences: no gate product exists) is held to TOL of dv's RMS instead."""
+    floor = np.sqrt(np.mean(ref["v"] ** 2))
+    for n in NAMES:
+        assert np.isfinite(got[n]).all(), f"d{n} left unwritten"
+        rms = np.sqrt(np.mean(ref[n] ** 2)) if ref[n].size else 0.0
+        err = np.max(np.abs(got[n] - ref[n])) / max(rms, floor) if ref[n].size else 0.0
+        assert err <= TOL, f"d{n}: rel max err {err:.3e}"
+
+
+def _do(inp, seed):
+    do = np.random.default_rng(seed).standard_normal(inp.v.shape).astype(np.float32)
+    return I.round_to_bf16(do) if inp.dtype == "bf16" else do
+
+
+CASES = {
+    "t256_d32_f32": (I.shrink(W["t256_d32_f32"], B=1, H=2, T=256), "dist"),
+    "t300_d64_bf16_slow": (I.shrink(W["t2k_d64_bf16"], B=2, H=3, T=300), "slow"),
+    "t2k_d64_bf16": (I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=2048), "slow"),
+    "t1_d64_bf16": (I.shrink(W["t2k_d64_bf16"], B=2, H=1, T=1), "dist"),
+    "t33_d32_f32": (I.shrink(W["t256_d32_f32"], B=2, H=1, T=33), "slow"),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_matches_oracle(name):
+    w, mode = CASES[name]
+    inp = I.make_inputs(w, seed=21, log_a_mode=mode)
+    do = _do(inp, 22)
+    _check(_run(inp, do), O.llattn_backward(inp, do))
+
+
+def test_backward_packed_sequences():
+    w = I.shrink(W["varlen8_d64_bf16"], B=4, H=2, T=600, len_lo=0, len_hi=600)
+    inp = I.make_inputs(w, seed=23, log_a_mode="slow", lengths=np.array([317, 0, 1, 600]))
+    do = _do(inp, 24)
+    _check(_run(inp, do), O.llattn_backward(inp, do))
+
+
+def test_backward_one_hot_deep_level():
+    """Only level 11 weighted: the top blocks' rank-d interaction alone carries dq, dk, dv."""
+    w = I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=2048)
+    inp = I.make_inputs(w, seed=25, log_a_mode="slow", lam_mode="onehot", lam_level=11)
+    do = _do(inp, 26)
+    _check(_run(inp, do), O.llattn_backward(inp, do))
+
+
+def test_backward_at_the_benchmark_size_sampled():
+    """B=4, H=32, T=8192, d=64 (the benchmark's launch configuration): 48 sampled (token,
+    head) rows and columns against the oracle's direct sums, and every gradient finite."""
+    inp = I.make_inputs(W["t8k_d64_bf16"], seed=27)
+    do = _do(inp, 28)
+    got = _run(inp, do)
+    for n in NAMES:
+        assert np.isfinite(got[n]).all(), f"{n} left unwritten"
+    rng = np.random.default_rng(29)
+    total = inp.total_tokens
+    toks = np.concatenate([[0, 1, 8191, 4096, 8192, total - 1], rng.integers(0, total, 42)])
+    samples = [(int(t), int(h)) for t, h in zip(toks, rng.integers(0, inp.H, len(toks)))]
+    ref = O.llattn_backward_sampled(inp, do, samples)
+    for n in ("q", "k", "v", "lam"):
+        g = got[n].reshape(total, inp.H, -1)
+        mine = np.array([g[t, h] for t, h in samples])
+        err = O.rel_max_err(mine, ref[n])
+        assert err <= TOL, f"d{n}: rel max err {err:.3e}"
