@@ -26,7 +26,7 @@
 // Kernels, in stream order: the prefix sums g (fp64: the differences of long prefix sums must
 // stay exact), the dense tiles (they initialise dq, dk, dv and dlam[:, 0..5]), one launch per
 // level 6..L-1 (each token sits in one block per level, so the updates of one launch never
-// collide), and the reverse scan for dlog_a.  Arithmetic is fp32 on CUDA cores; d = dk = dv in
+// collide), then dg per (token, head) and its reverse scan for dlog_a.  Arithmetic is fp32 on CUDA cores; d = dk = dv in
 // {32, 64}.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dense_tile(BwdProblem p, const d
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kThreads) bwd_level_block(BwdProblem p, const double* g, int lvl) {
   constexpr int R = D * D / kThreads;  // state elements per thread
-  constexpr int W = D / 32;            // outputs per lane in the per-token products
+  constexpr int E = D / 8;             // elements per lane of an 8-lane token group
   __shared__ float s_mem[2 * D * (D + 1)];  // phase 1: staged rows; phase 2: S and U
   __shared__ float s_w[32];
   float (*s_x)[D] = reinterpret_cast<float (*)[D]>(s_mem);               // [32][D]
@@ -237,95 +237,121 @@ __global__ void __launch_bounds__(kThreads) bwd_level_block(BwdProblem p, const 
   }
   __syncthreads();
 
-  // phase 2, right half (one warp per token): w = e^{g_t - g_m} S do_t; dlam; dq
-  for (int t = mid + warp; t < rend; t += kThreads / 32) {
-    const size_t rr = row(t);
-    float dol[W], ql[W], wl[W];
+  // phase 2: 32 tokens per pass, four per warp, one 8-lane group per token.  Lane j of a group
+  // owns elements j, j+8, j+16, ... (E of them), so the 8 lanes read 8 consecutive words of a
+  // state row (no bank conflicts), and the element b of the token's vector that a product needs
+  // comes from lane b % 8 of the group, register b / 8.
+  const int grp = lane >> 3, j = lane & 7, src0 = lane & ~7;
+  // right half: w = e^{g_t - g_m} S do_t;  dlam[t, l] = q_t . w;  dq_t += lam[t, l] w
+  for (int base = mid; base < rend; base += 32) {
+    const int t = base + warp * 4 + grp;
+    const bool ok = t < rend;
+    const size_t rr = ok ? row(t) : 0;
+    float xd[E], xq[E], w[E];
 #pragma unroll
-    for (int u = 0; u < W; ++u) {
-      dol[u] = ld_in(dout + rr * D + lane + 32 * u);
-      ql[u] = ld_in(q + rr * D + lane + 32 * u);
-      wl[u] = 0.f;
+    for (int m = 0; m < E; ++m) {
+      xd[m] = ok ? ld_in(dout + rr * D + j + 8 * m) : 0.f;
+      xq[m] = ok ? ld_in(q + rr * D + j + 8 * m) : 0.f;
+      w[m] = 0.f;
     }
 #pragma unroll
-    for (int u2 = 0; u2 < W; ++u2)
-      for (int bb = 0; bb < 32; ++bb) {
-        const float dob = __shfl_sync(kFull, dol[u2], bb);
-        const int b = bb + 32 * u2;
+    for (int b = 0; b < D; ++b) {
+      const float db = __shfl_sync(kFull, xd[b >> 3], src0 | (b & 7));
 #pragma unroll
-        for (int u = 0; u < W; ++u) wl[u] = fmaf(s_S[lane + 32 * u][b], dob, wl[u]);
-      }
-    const float sc = expf((float)(g[grow(t)] - gm));
-    const float lam = p.lam[rr * p.L + lvl];
+      for (int m = 0; m < E; ++m) w[m] = fmaf(s_S[j + 8 * m][b], db, w[m]);
+    }
+    const float sc = ok ? expf((float)(g[grow(ok ? t : mid)] - gm)) : 0.f;
+    const float lam = ok ? p.lam[rr * p.L + lvl] : 0.f;
     float dl = 0.f;
 #pragma unroll
-    for (int u = 0; u < W; ++u) {
-      wl[u] *= sc;
-      dl = fmaf(ql[u], wl[u], dl);
-      p.dq[rr * D + lane + 32 * u] += lam * wl[u];
+    for (int m = 0; m < E; ++m) {
+      w[m] *= sc;
+      dl = fmaf(xq[m], w[m], dl);
     }
+    dl += __shfl_xor_sync(kFull, dl, 1);
+    dl += __shfl_xor_sync(kFull, dl, 2);
+    dl += __shfl_xor_sync(kFull, dl, 4);
+    if (ok) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dl += __shfl_xor_sync(kFull, dl, off);
-    if (lane == 0) p.dlam[rr * p.L + lvl] = dl;
+      for (int m = 0; m < E; ++m) p.dq[rr * D + j + 8 * m] += lam * w[m];
+      if (j == 0) p.dlam[rr * p.L + lvl] = dl;
+    }
   }
-
-  // phase 2, left half: dk_s += e^{g_m - g_s} U v_s, dv_s += e^{g_m - g_s} U^T k_s
-  for (int s = lo + warp; s < lend; s += kThreads / 32) {
-    const size_t rr = row(s);
-    float vl[W], kl[W], ak[W], av[W];
+  // left half: dk_s += e^{g_m - g_s} U v_s;  dv_s += e^{g_m - g_s} U^T k_s
+  for (int base = lo; base < lend; base += 32) {
+    const int s = base + warp * 4 + grp;
+    const bool ok = s < lend;
+    const size_t rr = ok ? row(s) : 0;
+    float xv[E], xk[E], ak[E], av[E];
 #pragma unroll
-    for (int u = 0; u < W; ++u) {
-      vl[u] = ld_in(v + rr * D + lane + 32 * u);
-      kl[u] = ld_in(k + rr * D + lane + 32 * u);
-      ak[u] = av[u] = 0.f;
+    for (int m = 0; m < E; ++m) {
+      xv[m] = ok ? ld_in(v + rr * D + j + 8 * m) : 0.f;
+      xk[m] = ok ? ld_in(k + rr * D + j + 8 * m) : 0.f;
+      ak[m] = av[m] = 0.f;
     }
 #pragma unroll
-    for (int u2 = 0; u2 < W; ++u2)
-      for (int bb = 0; bb < 32; ++bb) {
-        const int b = bb + 32 * u2;
-        const float vb = __shfl_sync(kFull, vl[u2], bb);
-        const float kb = __shfl_sync(kFull, kl[u2], bb);
+    for (int b = 0; b < D; ++b) {
+      const float vb = __shfl_sync(kFull, xv[b >> 3], src0 | (b & 7));
+      const float kb = __shfl_sync(kFull, xk[b >> 3], src0 | (b & 7));
 #pragma unroll
-        for (int u = 0; u < W; ++u) {
-          ak[u] = fmaf(s_U[lane + 32 * u][b], vb, ak[u]);   // (U v)[a],   a = lane + 32u
-          av[u] = fmaf(s_U[b][lane + 32 * u], kb, av[u]);   // (U^T k)[c], c = lane + 32u
-        }
+      for (int m = 0; m < E; ++m) {
+        ak[m] = fmaf(s_U[j + 8 * m][b], vb, ak[m]);   // (U v)[a],   a = j + 8m
+        av[m] = fmaf(s_U[b][j + 8 * m], kb, av[m]);   // (U^T k)[c], c = j + 8m
       }
-    const float sc = expf((float)(gm - g[grow(s)]));
+    }
+    if (ok) {
+      const float sc = expf((float)(gm - g[grow(s)]));
 #pragma unroll
-    for (int u = 0; u < W; ++u) {
-      p.dk[rr * D + lane + 32 * u] += sc * ak[u];
-      p.dv[rr * D + lane + 32 * u] += sc * av[u];
+      for (int m = 0; m < E; ++m) {
+        p.dk[rr * D + j + 8 * m] += sc * ak[m];
+        p.dv[rr * D + j + 8 * m] += sc * av[m];
+      }
     }
   }
 }
 
-// ---- dlog_a: reverse prefix sums of dg_t = q_t . dq_t - k_t . dk_t, one warp each ----
+// ---- dlog_a: dg_t = q_t . dq_t - k_t . dk_t per (token, head), one warp each, into dlog_a ----
 template <typename Tin, int D>
-__global__ void bwd_dlog_a(BwdProblem p) {
-  const int h = blockIdx.x, sq = blockIdx.y, lane = threadIdx.x;
+__global__ void __launch_bounds__(kThreads) bwd_dg(BwdProblem p) {
+  const int h = blockIdx.y, sq = blockIdx.z, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
   const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  if (t >= sp.len) return;
   const Tin* q = static_cast<const Tin*>(p.q);
   const Tin* k = static_cast<const Tin*>(p.k);
-  double carry = 0.0;
-  for (int end = sp.len; end > 0; end -= 32) {
-    const int t = end - 32 + lane;
-    double x = 0.0;
-    if (t >= 0) {
-      const size_t rr = (size_t)(sp.start + t) * p.H + h;
-      float a = 0.f;
-      for (int c = 0; c < D; ++c)
-        a += ld_in(q + rr * D + c) * p.dq[rr * D + c] - ld_in(k + rr * D + c) * p.dk[rr * D + c];
-      x = a;
-    }
+  const size_t rr = (size_t)(sp.start + t) * p.H + h;
+  float a = 0.f;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const double y = __shfl_down_sync(kFull, x, off);
-      if (lane + off < 32) x += y;
-    }
-    x += carry;
-    if (t >= 0) p.dlog_a[(size_t)(sp.start + t) * p.H + h] = (float)x;
-    carry = __shfl_sync(kFull, x, 0);
+  for (int c = lane; c < D; c += 32)
+    a += ld_in(q + rr * D + c) * p.dq[rr * D + c] - ld_in(k + rr * D + c) * p.dk[rr * D + c];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(kFull, a, off);
+  if (lane == 0) p.dlog_a[rr] = a;
+}
+
+// ---- dlog_a[r] = sum over t >= r of dg_t, in place, one CTA per (sequence, head) ----
+__global__ void __launch_bounds__(kThreads) bwd_suffix_scan(BwdProblem p) {
+  __shared__ double s_part[kThreads];
+  const int h = blockIdx.x, sq = blockIdx.y, tid = threadIdx.x;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  const int seg = (sp.len + kThreads - 1) / kThreads;
+  const int t0 = min(tid * seg, sp.len), t1 = min(t0 + seg, sp.len);
+  float* x = p.dlog_a + (size_t)sp.start * p.H + h;   // token t at x[t * H]
+  double sum = 0.0;
+  for (int t = t0; t < t1; ++t) sum += x[(size_t)t * p.H];
+  s_part[tid] = sum;
+  __syncthreads();
+  // suffix sums of the per-thread totals (Hillis-Steele, reading the later entries)
+  for (int off = 1; off < kThreads; off <<= 1) {
+    const double y = tid + off < kThreads ? s_part[tid + off] : 0.0;
+    __syncthreads();
+    s_part[tid] += y;
+    __syncthreads();
+  }
+  double run = tid + 1 < kThreads ? s_part[tid + 1] : 0.0;  // everything after this segment
+  for (int t = t1 - 1; t >= t0; --t) {
+    run += x[(size_t)t * p.H];
+    x[(size_t)t * p.H] = (float)run;
   }
 }
 
@@ -339,8 +365,10 @@ cudaError_t launch(const BwdProblem& p, double* g, cudaStream_t st) {
     const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
     bwd_level_block<Tin, D><<<dim3(nblk, p.H, p.nseq), kThreads, 0, st>>>(p, g, lvl);
   }
-  bwd_dlog_a<Tin, D><<<seqs, 32, 0, st>>>(p);
-  count_launch(n + 1);
+  bwd_dg<Tin, D><<<dim3((p.T + kThreads / 32 - 1) / (kThreads / 32), p.H, p.nseq), kThreads, 0,
+                   st>>>(p);
+  bwd_suffix_scan<<<seqs, kThreads, 0, st>>>(p);
+  count_launch(n + 2);
   return cudaGetLastError();
 }
 
