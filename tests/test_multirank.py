@@ -48,8 +48,13 @@ def _worker(rank, world, port, q):
             steps, warmup, seed = 1, 0, 0
 
         ref_line = bench.run_reference(Args, I.shrink(w, T=32), rank, world)
+        # the backward and decoding benches' reference arms follow the same rule
+        bwd_line = bench.run_bwd_reference(Args, I.shrink(w, T=32), rank, world)
+        dw = I.DecodeWorkload("d", B=2, H=2, L=6, dk=32, dv=32, dtype="f32")
+        dec_line = bench.run_decode_reference(Args, dw, rank, world)
+        others = [x is None for x in (bwd_line, dec_line)]
         dist.barrier()
-        q.put((rank, worst, digests, ref_line is None, ref_line and ref_line["impl"]))
+        q.put((rank, worst, digests, ref_line is None, ref_line and ref_line["impl"], others))
     finally:
         dist.destroy_process_group()
 
@@ -64,8 +69,8 @@ def test_two_gloo_ranks():
         p.start()
     res = {}
     for _ in range(world):
-        rank, worst, digests, ref_none, impl = q.get(timeout=120)
-        res[rank] = (worst, digests, ref_none, impl)
+        rank, worst, digests, ref_none, impl, others = q.get(timeout=120)
+        res[rank] = (worst, digests, ref_none, impl, others)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -76,6 +81,7 @@ def test_two_gloo_ranks():
     # the reference arm prints on rank 0 only; other ranks do no work
     assert res[0][2] is False and res[0][3] == "reference"
     assert res[1][2] is True
+    assert res[0][4] == [False, False] and res[1][4] == [True, True]
 
 
 def test_single_process_helpers():
