@@ -254,7 +254,7 @@ LLATTN_API llattn_status llattn_fwd_noalloc(int in_dtype, const void* q, const v
  *             Read only: the caller advances it for the next step.  Setting pos[b] = 0 starts
  *             sequence b afresh; nothing else in the state has to be reset or cleared.
  *   state     DEVICE fp32 buffer of llattn_decode_state_bytes(), caller-owned and kept
- *             between steps.  Layout: levels [B, H, L-1, dk, dv] (slot j = level j+1, row-major
+ *             between steps (non-NULL even when that size is 0, i.e. L = 1).  Layout: levels [B, H, L-1, dk, dv] (slot j = level j+1, row-major
  *             dk x dv), then gate [B, H, 2, L-1].  A slot holds its level's state as it was
  *             when written; gate[b, h, p, j] is the log of the gate product slot j has missed
  *             since then, valid at positions of parity p.  The level's state just before
