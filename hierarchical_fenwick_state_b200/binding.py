@@ -23,7 +23,7 @@ EXPORTS = (
     "llattn_fwd_f32", "llattn_workspace_bytes", "llattn_fwd_ex", "llattn_device_status",
     "llattn_last_cuda_error", "llattn_fwd_host", "llattn_profile", "llattn_profile_read",
     "llattn_fwd_noalloc", "llattn_decode_state_bytes", "llattn_decode_step",
-    "llattn_bwd_workspace_bytes", "llattn_bwd",
+    "llattn_bwd_workspace_bytes", "llattn_bwd", "llattn_fwd_bf16", "llattn_stream_status",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20  # LLATTN_NOALLOC_SCRATCH_BYTES
@@ -80,6 +80,10 @@ def lib():
     L.llattn_bwd.restype = i
     L.llattn_bwd.argtypes = [i, vp, vp, vp, f_p, f_p, vp, f_p, f_p, f_p, f_p, f_p, i, i, i, i, i,
                              i_p, vp, ctypes.c_size_t, vp]
+    L.llattn_fwd_bf16.restype = i
+    L.llattn_fwd_bf16.argtypes = [vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_stream_status.restype = i
+    L.llattn_stream_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i, vp]
     L.llattn_profile.restype = i
     L.llattn_profile.argtypes = [i]
     L.llattn_profile_read.restype = i
@@ -168,6 +172,18 @@ def fwd(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None, stream=None)
                           ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None,
                           _stream_handle(stream))
     _check(st, "llattn_fwd")
+    return out
+
+
+def fwd_bf16(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens=None, stream=None):
+    """Direct call of llattn_fwd_bf16 (the same call as llattn_fwd)."""
+    st = lib().llattn_fwd_bf16(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                               ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(log_a.data_ptr()),
+                               ctypes.c_void_p(lam.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                               int(B), int(H), int(T), int(dk), int(dv),
+                               ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None,
+                               _stream_handle(stream))
+    _check(st, "llattn_fwd_bf16")
     return out
 
 
@@ -301,4 +317,13 @@ def device_status(clear: bool = True) -> int:
     st = lib().llattn_device_status(ctypes.byref(flags), int(clear))
     if st not in (0, 6):
         _check(st, "llattn_device_status")
+    return int(flags.value)
+
+
+def stream_status(clear: bool = True, stream=None) -> int:
+    """llattn_stream_status: the status word, read in order on one stream (no device sync)."""
+    flags = ctypes.c_uint(0)
+    st = lib().llattn_stream_status(ctypes.byref(flags), int(clear), _stream_handle(stream))
+    if st not in (0, 6):
+        _check(st, "llattn_stream_status")
     return int(flags.value)

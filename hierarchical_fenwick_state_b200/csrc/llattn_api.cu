@@ -33,6 +33,7 @@ struct DeviceState {
 
 std::mutex g_mu;
 std::mutex g_host_mu;
+std::mutex g_status_mu;   // lazy per-device lookup of the status word's address
 DeviceState g_dev[kMaxDevices];
 
 llattn_status cuda_fail(cudaError_t e) {
@@ -85,11 +86,14 @@ llattn_status device_state(DeviceState** out, int* dev_out) {
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return LLATTN_ERR_ARG;
   DeviceState& d = g_dev[dev];
-  if (d.status == nullptr) {
-    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_llattn_status);
-    if (e != cudaSuccess) {
-      d.status = nullptr;
-      return cuda_fail(e);
+  {
+    // first calls from several host threads look the address up once, under a lock
+    std::lock_guard<std::mutex> hold(g_status_mu);
+    if (d.status == nullptr) {
+      unsigned int* addr = nullptr;
+      e = cudaGetSymbolAddress(reinterpret_cast<void**>(&addr), g_llattn_status);
+      if (e != cudaSuccess) return cuda_fail(e);
+      d.status = addr;
     }
   }
   *out = &d;
@@ -299,6 +303,12 @@ llattn_status llattn_fwd(const void* q, const void* k, const void* v, const floa
                  cu_seqlens, nullptr, 0, stream);
 }
 
+llattn_status llattn_fwd_bf16(const void* q, const void* k, const void* v, const float* log_a,
+                              const float* lam, float* out, int B, int H, int T, int dk, int dv,
+                              const int* cu_seqlens, void* stream) {
+  return llattn_fwd(q, k, v, log_a, lam, out, B, H, T, dk, dv, cu_seqlens, stream);
+}
+
 llattn_status llattn_fwd_f32(const float* q, const float* k, const float* v, const float* log_a,
                              const float* lam, float* out, int B, int H, int T, int dk, int dv,
                              const int* cu_seqlens, void* stream) {
@@ -347,6 +357,27 @@ llattn_status llattn_device_status(unsigned int* flags, int clear) {
     return cuda_fail(e);
   if (clear && v) {
     if ((e = cudaMemset(ds->status, 0, sizeof(v))) != cudaSuccess) return cuda_fail(e);
+  }
+  *flags = v;
+  return (v & LLATTN_DEV_WAIT_TIMEOUT) ? LLATTN_ERR_TIMEOUT : LLATTN_OK;
+}
+
+llattn_status llattn_stream_status(unsigned int* flags, int clear, void* stream) {
+  if (!flags) return LLATTN_ERR_ARG;
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  llattn_status s = device_state(&ds, &dev);
+  if (s != LLATTN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // stream-ordered copy into a pageable word; the synchronise makes it complete
+  unsigned int v = 0;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(&v, ds->status, sizeof(v), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e);
+  if (clear && v) {
+    if ((e = cudaMemsetAsync(ds->status, 0, sizeof(unsigned int), st)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e);
   }
   *flags = v;
   return (v & LLATTN_DEV_WAIT_TIMEOUT) ? LLATTN_ERR_TIMEOUT : LLATTN_OK;

@@ -11,7 +11,8 @@
 // Query chunk c therefore reads one block state per set bit b of c: the 2^b
 // chunks just before the aligned 2^(b+1)-chunk group of c.  Those block states
 // form a binary counter over chunks (the recurrent form's "merge on promotion",
-// "Forma Ricorrente"), kept here in shared memory as bf16 hi/lo pairs.
+// "Forma Ricorrente"), kept here in shared memory (bf16 hi/lo pairs in the serial
+// cross-check, fp16 in the pipelined kernel).
 //
 // Per chunk (all five steps fused in this one kernel; the weighted readout over
 // levels is fused into the epilogue, as in "kernel ... que fusionan operaciones a
@@ -1012,6 +1013,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
 #pragma unroll
     for (int b = 0; b < kLevels; ++b) gtot[b] = 0.f;
     uint32_t u = 0;
+    // An fp16 operand out of range (|x| >= 65520 rounds to inf) reaches the output as inf
+    // or NaN, so checking every output value catches it; the host sees a status bit.
+    bool nonfinite = false;
     for (int c = 0; c < nch; ++c) {
       const int s = c % kPStages;
       const int n = min(kC, sp.len - c * kC);
@@ -1128,6 +1132,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           if (b == m) gtot[b] = acc;
         mbar_arrive(&bars[(c & 1) ? B_LV1 : B_LV]);
       }
+      if (row < n) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          nonfinite |= !(fabsf(o2[e].x) <= 3.402823466e38f) | !(fabsf(o2[e].y) <= 3.402823466e38f);
+      }
       if (n == kC) {
         // Whole chunk: stage the 128 x 64 fp32 tile in the Q (columns 0..31) and K (32..63)
         // tiles of this stage -- every reader of them is done by now -- in the 128-byte
@@ -1152,6 +1161,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
       mbar_arrive(&bars[B_GEMPTY + c % kPG]);
     }
+    if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(status, LLATTN_DEV_NONFINITE);
   } else {
     // ------------------------------------------------------------ inter-chunk MMA issuer
     // Per chunk c: the readout chains of the set bits of c (they need the level states left

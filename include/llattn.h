@@ -98,7 +98,12 @@ enum {
   LLATTN_DEV_SEQ_TOO_LONG = 1u,  /* a varlen sequence was longer than T */
   LLATTN_DEV_WAIT_TIMEOUT = 2u,  /* an mbarrier / pipeline wait hit its iteration limit */
   LLATTN_DEV_BAD_CU_SEQLENS = 4u, /* cu_seqlens decreasing */
-  LLATTN_DEV_DECODE_POS = 8u     /* llattn_decode_step: a position outside [0, 2^(L-1)) */
+  LLATTN_DEV_DECODE_POS = 8u,    /* llattn_decode_step: a position outside [0, 2^(L-1)) */
+  LLATTN_DEV_NONFINITE = 16u     /* tensor-core forward: an output value came out inf or NaN.
+                                  * With finite inputs this means an intermediate rounded to
+                                  * fp16 (P, V, the decay-scaled K, a level state, Q) left
+                                  * the fp16 range (|x| >= 65520): any such overflow reaches
+                                  * the output as inf or NaN.  Rerun on LLATTN_PATH_SIMT. */
 };
 
 /* Version of this ABI (increments on any signature change). */
@@ -122,6 +127,12 @@ LLATTN_API int llattn_num_levels(int T);
 LLATTN_API llattn_status llattn_fwd(const void* q, const void* k, const void* v, const float* log_a,
                          const float* lam, float* out, int B, int H, int T, int dk, int dv,
                          const int* cu_seqlens, void* stream);
+
+/* llattn_fwd_bf16 - the same call as llattn_fwd, named for its input type. */
+LLATTN_API llattn_status llattn_fwd_bf16(const void* q, const void* k, const void* v,
+                                         const float* log_a, const float* lam, float* out, int B,
+                                         int H, int T, int dk, int dv, const int* cu_seqlens,
+                                         void* stream);
 
 /* llattn_fwd_f32 - the same operation on fp32 q, k, v (CUDA-core fp32 path, no
  * tensor cores, so results meet a 1e-4 relative bound).  Arguments as llattn_fwd. */
@@ -158,6 +169,16 @@ LLATTN_API llattn_status llattn_fwd_ex(int in_dtype, int path, int chunk, const 
  * current device.  Synchronises the device.  *flags receives LLATTN_DEV_* bits.
  */
 LLATTN_API llattn_status llattn_device_status(unsigned int* flags, int clear);
+
+/*
+ * llattn_stream_status - the same read, ordered on one stream instead of the whole
+ * device: waits for the work already enqueued on `stream` (a cudaStream_t; NULL =
+ * legacy default stream), then copies the status word back (and clears it, if
+ * clear != 0) on that stream.  The word is per device, so it also holds bits set by
+ * kernels of other streams that have finished by then.  Returns LLATTN_ERR_TIMEOUT
+ * when LLATTN_DEV_WAIT_TIMEOUT is set, else LLATTN_OK (or a CUDA error).
+ */
+LLATTN_API llattn_status llattn_stream_status(unsigned int* flags, int clear, void* stream);
 
 /*
  * llattn_fwd_host - the forward on HOST buffers, for callers whose data is not
@@ -300,7 +321,9 @@ LLATTN_API llattn_status llattn_decode_step(int in_dtype, const void* q, const v
  *   q, k, v, log_a, lam, B, H, T, cu_seqlens   as in llattn_fwd.
  *   dout       [B, T, H, dv] (packed: [total, H, dv]), the gradient of the loss at out.
  *   dq, dk, dv [.., H, d] fp32; dlog_a [.., H] fp32; dlam [.., H, L] fp32: fully overwritten
- *              for every token of every sequence.
+ *              for every token of every sequence, with one exception: a packed sequence
+ *              longer than T is cut at T (as in the forward), its rows past T are left
+ *              unwritten, and LLATTN_DEV_SEQ_TOO_LONG is set in the device status word.
  *   workspace  caller-owned device scratch of llattn_bwd_workspace_bytes() bytes (256-byte
  *              aligned), or NULL for the library's per-device buffer (as llattn_fwd).
  * Pointers: q, k, v, dout, dq, dk, dv 16-byte aligned, the rest 4-byte aligned; no gradient

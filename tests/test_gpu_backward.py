@@ -90,7 +90,8 @@ def test_backward_one_hot_deep_level():
 
 def test_backward_at_the_benchmark_size_sampled():
     """B=4, H=32, T=8192, d=64 (the benchmark's launch configuration): 48 sampled (token,
-    head) rows and columns against the oracle's direct sums, and every gradient finite."""
+    head) rows and columns against the oracle's direct sums, dlog_a of two whole (sequence,
+    head) pairs against the oracle's full backward, and every gradient finite."""
     inp = I.make_inputs(W["t8k_d64_bf16"], seed=27)
     do = _do(inp, 28)
     got = _run(inp, do)
@@ -106,3 +107,16 @@ def test_backward_at_the_benchmark_size_sampled():
         mine = np.array([g[t, h] for t, h in samples])
         err = O.rel_max_err(mine, ref[n])
         assert err <= TOL, f"d{n}: rel max err {err:.3e}"
+    # dlog_a is a suffix sum over up to 8192 tokens, fed by every level down to the top two
+    # blocks: compare it in full, for two (sequence, head) pairs, with the oracle's whole
+    # backward of that sequence and head (about 9 s and 6 GB of fp64 each).
+    T = inp.T
+    for b, h in ((0, 5), (3, 30)):
+        sl = slice(b * T, (b + 1) * T)
+        f = {n: getattr(inp, n).reshape(total, inp.H, -1)[sl, h] for n in ("q", "k", "v", "lam")}
+        la = inp.log_a.reshape(total, inp.H)[sl, h]
+        dref = O.llattn_backward_seq(f["q"], f["k"], f["v"], la, f["lam"],
+                                     do.reshape(total, inp.H, -1)[sl, h])[3]
+        mine = got["log_a"].reshape(total, inp.H)[sl, h]
+        err = O.rel_max_err(mine, dref)
+        assert err <= TOL, f"dlog_a (sequence {b}, head {h}): rel max err {err:.3e}"

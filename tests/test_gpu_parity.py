@@ -221,3 +221,57 @@ def test_kernel_boundaries_odd_heads(T):
     ref = O.llattn_recurrent(inp)
     for path in _paths_for(inp):
         _check(inp, ref, path)
+
+
+# ------------------------------------------------------------------------------------------------
+# Range guard of the tensor-core path's fp16 operands, and the status word read per stream
+# ------------------------------------------------------------------------------------------------
+def test_fp16_range_guard_sets_status_bit():
+    """v scaled by 1e5 leaves the fp16 range on the tensor-core path (V, P V and the level
+    states are rounded to fp16 there): the output turns non-finite and the kernel sets
+    LLATTN_DEV_NONFINITE, read here through the per-stream status call.  The CUDA-core path
+    computes in fp32 and matches the oracle on the same inputs."""
+    import torch
+    w = I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=1000)
+    inp = I.make_inputs(w, seed=5)
+    inp.v = I.round_to_bf16(inp.v * np.float32(1e5))
+    ref = O.llattn_recurrent(inp)
+    t = _to_device_for_guard(inp)
+    out = torch.empty(inp.v.shape, dtype=torch.float32, device="cuda:0")
+    binding.stream_status(clear=True)
+    binding.forward(t["q"], t["k"], t["v"], t["log_a"], t["lam"], T=inp.T, out=out,
+                    path="tcgen05")
+    flags = binding.stream_status(clear=True)
+    assert flags & 16, f"LLATTN_DEV_NONFINITE not set (flags {flags})"
+    assert not np.isfinite(out.double().cpu().numpy()).all()
+    out.fill_(float("nan"))
+    binding.forward(t["q"], t["k"], t["v"], t["log_a"], t["lam"], T=inp.T, out=out, path="simt")
+    assert binding.stream_status(clear=True) == 0
+    got = out.double().cpu().numpy()
+    assert O.rel_max_err(got, ref) <= TOL["bf16"]
+    # in-range inputs leave the bit clear on the tensor-core path
+    inp2 = I.make_inputs(w, seed=5)
+    t2 = _to_device_for_guard(inp2)
+    binding.forward(t2["q"], t2["k"], t2["v"], t2["log_a"], t2["lam"], T=inp2.T, out=out,
+                    path="tcgen05")
+    assert binding.stream_status(clear=True) == 0
+
+
+def _to_device_for_guard(inp):
+    from _llattn_cases import to_device
+    return to_device(inp)
+
+
+def test_fwd_bf16_alias_matches_fwd():
+    import torch
+    w = I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=700)
+    inp = I.make_inputs(w, seed=6)
+    t = _to_device_for_guard(inp)
+    o1 = torch.full(inp.v.shape, float("nan"), dtype=torch.float32, device="cuda:0")
+    o2 = torch.full_like(o1, float("nan"))
+    args = (t["q"], t["k"], t["v"], t["log_a"], t["lam"])
+    binding.fwd(*args, o1, inp.B, inp.H, inp.T, inp.dk, inp.dv)
+    binding.fwd_bf16(*args, o2, inp.B, inp.H, inp.T, inp.dk, inp.dv)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    assert binding.stream_status(clear=True) == 0
