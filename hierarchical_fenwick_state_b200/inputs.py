@@ -122,6 +122,7 @@ class Inputs:
     dk: int
     dv: int
     dtype: str
+    beta: Optional[np.ndarray] = None   # write strength of the gated delta rule, [..., H]
 
     @property
     def L(self) -> int:
@@ -203,6 +204,30 @@ def make_inputs(w: Workload, seed: int = 0, *, log_a_mode: str = "dist",
                   log_a=np.ascontiguousarray(log_a, np.float32),
                   lam=np.ascontiguousarray(lam, np.float32), cu_seqlens=cu,
                   B=B, H=H, T=w.T, dk=dk, dv=dv, dtype=w.dtype)
+
+
+def _sigmoid(x: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def make_gdn_inputs(w: Workload, seed: int = 0, *, beta_mode: str = "dist",
+                    **kw) -> Inputs:
+    """The inputs of ``make_inputs`` (same seed, same draws; log_a is the gate log alpha) plus
+    the delta rule's write strength beta per (token, head), from its own seeded stream:
+    "dist" sigmoid(N(0, 1)), "ones" (beta = 1) or "zero"."""
+    inp = make_inputs(w, seed, **kw)
+    lead = inp.log_a.shape
+    if beta_mode == "dist":
+        z = np.random.default_rng(seed + 104729).standard_normal(lead, dtype=np.float32)
+        beta = _sigmoid(z.astype(np.float64)).astype(np.float32)
+    elif beta_mode == "ones":
+        beta = np.ones(lead, np.float32)
+    elif beta_mode == "zero":
+        beta = np.zeros(lead, np.float32)
+    else:
+        raise ValueError(beta_mode)
+    inp.beta = np.ascontiguousarray(beta)
+    return inp
 
 
 def make_patterned(T: int, *, H: int = 1, dk: int = 64, dv: int = 64, log_a: float = 0.0,

@@ -11,3 +11,7 @@ from .llattn_oracle import (  # noqa: F401
     llattn_level_states, llattn_decode_step, llattn_decode_sequence, llattn_decode_batch,
     llattn_backward_seq, llattn_backward, llattn_backward_sampled,
 )
+from .gdn_oracle import (  # noqa: F401
+    gdn_bruteforce_seq, gdn_recurrent_seq, gated_deltanet_seq, gdn_single,
+    gdn_recurrent, gdn_bruteforce, gated_deltanet, gdn_sampled,
+)
