@@ -268,20 +268,123 @@ def oracle_sample_rate(inp, heads, seconds_hint=None):
     return rate, desc, dt
 
 
+def _oracle_head_worker(arrs):
+    """One head of the recurrent fp64 oracle in a worker process (single-threaded BLAS)."""
+    import oracle as O
+    t0 = time.perf_counter()
+    O.llattn_recurrent_seq(*arrs)
+    return time.perf_counter() - t0
+
+
+def _host_info():
+    info = {"cpu_count": os.cpu_count()}
+    try:
+        from threadpoolctl import threadpool_info
+        blas = [d for d in threadpool_info() if d.get("user_api") == "blas"]
+        info["blas_threads"] = int(sum(d.get("num_threads", 0) for d in blas)) if blas else None
+    except Exception:  # noqa: BLE001
+        info["blas_threads"] = None
+    return info
+
+
+class OraclePool:
+    """Worker processes for the recurrent fp64 oracle, one head per task, each with a
+    single-threaded BLAS (spawn context: safe after CUDA has been initialised)."""
+
+    def __init__(self, cores=None):
+        import multiprocessing as mp
+        self.cores = max(1, cores or os.cpu_count() or 1)
+        keep = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS",
+                                                "MKL_NUM_THREADS")}
+        for k in keep:
+            os.environ[k] = "1"          # inherited by the spawned workers
+        try:
+            self.pool = mp.get_context("spawn").Pool(self.cores)
+        finally:
+            for k, v in keep.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+    def rate(self, inp):
+        """Every head of the first sequence, spread over the cores; returns (tok/s of the
+        whole workload, cores used, description, wall seconds)."""
+        import numpy as np
+        start, n = inp.seq_slices()[0]
+        sl = slice(start, start + n)
+
+        def head(h, m=None):
+            e = sl if m is None else slice(start, start + m)
+            return (np.ascontiguousarray(inp.q.reshape(-1, inp.H, inp.dk)[e, h][None]),
+                    np.ascontiguousarray(inp.k.reshape(-1, inp.H, inp.dk)[e, h][None]),
+                    np.ascontiguousarray(inp.v.reshape(-1, inp.H, inp.dv)[e, h][None]),
+                    np.ascontiguousarray(inp.log_a.reshape(-1, inp.H)[e, h][None]),
+                    np.ascontiguousarray(inp.lam.reshape(-1, inp.H, inp.L)[e, h][None]))
+
+        # every worker started (imports done) before the clock: a tiny task each
+        self.pool.map(_oracle_head_worker, [head(0, min(n, 8))] * self.cores)
+        work = [head(h) for h in range(inp.H)]
+        used = min(self.cores, inp.H)
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_head_worker, work, chunksize=1)
+        wall = time.perf_counter() - t0
+        desc = (f"recurrent fp64 oracle form, 1 sequence x all {inp.H} heads x {n} tokens, one "
+                f"head per task on {used} host cores (spawned pool, single-threaded BLAS each), "
+                f"{wall:.2f} s wall")
+        return n / wall, used, desc, wall
+
+
+def oracle_allcores_rate(inp):
+    pool = OraclePool()
+    try:
+        return pool.rate(inp)
+    finally:
+        pool.close()
+
+
+def oracle_quadratic_rate(inp, max_tokens=4096):
+    """The quadratic (masked) fp64 oracle form on one head of the first sequence's first
+    `max_tokens` tokens, with the process's BLAS threads; tok/s of the workload at that
+    prefix length (the form's cost grows with T^2, so the full length is slower still)."""
+    import numpy as np
+    import oracle as O
+    start, n = inp.seq_slices()[0]
+    m = min(n, max_tokens)
+    sl = slice(start, start + m)
+    t0 = time.perf_counter()
+    O.llattn_quadratic_seq(inp.q.reshape(-1, inp.H, inp.dk)[sl, 0],
+                           inp.k.reshape(-1, inp.H, inp.dk)[sl, 0],
+                           inp.v.reshape(-1, inp.H, inp.dv)[sl, 0],
+                           inp.log_a.reshape(-1, inp.H)[sl, 0],
+                           inp.lam.reshape(-1, inp.H, inp.L)[sl, 0])
+    dt = time.perf_counter() - t0
+    return {"value": m / inp.H / dt, "unit": "tokens/s", "kind": "oracle (quadratic form)",
+            "sample": f"1 head x first {m} tokens of one sequence, {dt:.2f} s, BLAS threads of "
+                      f"the process; cost grows as T^2"}
+
+
 def run_reference(args, w, rank, world):
     """The oracle as it stands, timed on the host cores (rank 0 only)."""
     from hierarchical_fenwick_state_b200 import inputs as I
     if rank != 0:
         return None
     inp = I.make_inputs(w, seed=args.seed)
-    heads = 1
-    for _ in range(args.warmup):
-        oracle_sample_rate(inp, heads)
-    times, rates = [], []
-    for _ in range(args.steps):
-        r, desc, dt = oracle_sample_rate(inp, heads)
-        times.append(dt)
-        rates.append(r)
+    pool = OraclePool()
+    try:
+        for _ in range(args.warmup):
+            oracle_sample_rate(inp, 1)
+        times, rates = [], []
+        for _ in range(args.steps):
+            r, cores, desc, dt = pool.rate(inp)
+            times.append(dt)
+            rates.append(r)
+    finally:
+        pool.close()
     value = float(statistics.mean(rates))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -290,8 +393,8 @@ def run_reference(args, w, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
         "config": workload_config(w, None, None),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": desc + " per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc + " per step", "host": _host_info()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -481,9 +584,10 @@ def run_ours(args, w, rank, world, local_rank):
                        "steps": n_e2e, "entry": "llattn_fwd_host (pinned host buffers)"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, _ = oracle_sample_rate(inp, heads=min(inp.H, 12))
-        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": desc}
+        rate, cores, desc, _ = oracle_allcores_rate(inp)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": desc, "host": _host_info(),
+                                "quadratic_form": oracle_quadratic_rate(inp)}
     return line
 
 

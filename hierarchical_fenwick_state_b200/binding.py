@@ -24,6 +24,7 @@ EXPORTS = (
     "llattn_last_cuda_error", "llattn_fwd_host", "llattn_profile", "llattn_profile_read",
     "llattn_fwd_noalloc", "llattn_decode_state_bytes", "llattn_decode_step",
     "llattn_bwd_workspace_bytes", "llattn_bwd", "llattn_fwd_bf16", "llattn_stream_status",
+    "llattn_segment_plan", "llattn_set_segment_chunks", "llattn_gdn_fwd",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20  # LLATTN_NOALLOC_SCRATCH_BYTES
@@ -84,6 +85,12 @@ def lib():
     L.llattn_fwd_bf16.argtypes = [vp, vp, vp, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
     L.llattn_stream_status.restype = i
     L.llattn_stream_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i, vp]
+    L.llattn_gdn_fwd.restype = i
+    L.llattn_gdn_fwd.argtypes = [i, vp, vp, vp, f_p, f_p, f_p, f_p, i, i, i, i, i, i_p, vp]
+    L.llattn_segment_plan.restype = i
+    L.llattn_segment_plan.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int)]
+    L.llattn_set_segment_chunks.restype = i
+    L.llattn_set_segment_chunks.argtypes = [i]
     L.llattn_profile.restype = i
     L.llattn_profile.argtypes = [i]
     L.llattn_profile_read.restype = i
@@ -318,6 +325,49 @@ def device_status(clear: bool = True) -> int:
     if st not in (0, 6):
         _check(st, "llattn_device_status")
     return int(flags.value)
+
+
+def gdn_forward(q, k, v, log_alpha, beta, lam, *, cu_seqlens=None, T: Optional[int] = None,
+                out=None, stream=None):
+    """Log-Linear Gated DeltaNet forward (llattn_gdn_fwd) on device tensors; returns out (fp32).
+    Layouts as ``forward``; log_alpha and beta are [.., H] fp32."""
+    import torch
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q/k/v must be bf16 or fp32")
+    for t in (q, k, v, log_alpha, beta, lam):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    H, dk, dv = q.shape[-2], q.shape[-1], v.shape[-1]
+    if cu_seqlens is None:
+        B, T = q.shape[0], q.shape[1]
+    else:
+        B = cu_seqlens.numel() - 1
+        if T is None:
+            raise ValueError("packed inputs need T (the bound on every length)")
+    if out is None:
+        out = torch.empty(v.shape, dtype=torch.float32, device=v.device)
+    in_dtype = BF16 if q.dtype == torch.bfloat16 else F32
+    cu_ptr = ctypes.c_void_p(cu_seqlens.data_ptr()) if cu_seqlens is not None else None
+    st = lib().llattn_gdn_fwd(in_dtype, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                              ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(log_alpha.data_ptr()),
+                              ctypes.c_void_p(beta.data_ptr()), ctypes.c_void_p(lam.data_ptr()),
+                              ctypes.c_void_p(out.data_ptr()), int(B), int(H), int(T), int(dk),
+                              int(dv), cu_ptr, _stream_handle(stream))
+    _check(st, "llattn_gdn_fwd")
+    return out
+
+
+def segment_plan(B: int, H: int, T: int, dk: int, dv: int, varlen: bool = False) -> int:
+    """Chunks per segment of a tensor-core call of this shape (0: whole sequences per CTA)."""
+    n = ctypes.c_int(0)
+    _check(lib().llattn_segment_plan(B, H, T, dk, dv, int(varlen), ctypes.byref(n)),
+           "llattn_segment_plan")
+    return int(n.value)
+
+
+def set_segment_chunks(chunks: int) -> None:
+    """Force the tensor-core path's segment length (0: automatic)."""
+    _check(lib().llattn_set_segment_chunks(int(chunks)), "llattn_set_segment_chunks")
 
 
 def stream_status(clear: bool = True, stream=None) -> int:

@@ -10,6 +10,7 @@
 #include "../../include/llattn.h"
 #include "llattn_bwd.h"
 #include "llattn_decode.h"
+#include "llattn_gdn.h"
 #include "llattn_internal.h"
 
 // Per-device status word: kernels OR LLATTN_DEV_* bits into it.
@@ -75,9 +76,9 @@ llattn_status resolve(int in_dtype, int* path, int* chunk, int T, int dk, int dv
   return LLATTN_OK;
 }
 
-size_t workspace_for(int path, int chunk, int nseq, int H, int T, int dk, int dv) {
+size_t workspace_for(int path, int chunk, int nseq, int H, int T, int dk, int dv, bool varlen) {
   if (path == LLATTN_PATH_SIMT) return llattn::simt_workspace_bytes(nseq, H, T, dk, dv, chunk);
-  return llattn::tc_workspace_bytes(nseq, H, T, dk, dv, chunk);
+  return llattn::tc_workspace_bytes(nseq, H, T, dk, dv, chunk, varlen);
 }
 
 llattn_status device_state(DeviceState** out, int* dev_out) {
@@ -165,7 +166,7 @@ llattn_status forward(int in_dtype, int path, int chunk, const void* q, const vo
   DeviceState* ds = nullptr;
   int dev = 0;
   if ((s = device_state(&ds, &dev)) != LLATTN_OK) return s;
-  const size_t need = workspace_for(path, chunk, B, H, T, dk, dv);
+  const size_t need = workspace_for(path, chunk, B, H, T, dk, dv, cu_seqlens != nullptr);
   void* ws = workspace;
   std::unique_lock<std::mutex> lock(g_mu, std::defer_lock);
   if ((s = pick_workspace(ds, need, workspace, workspace_bytes, lock, &ws)) != LLATTN_OK) return s;
@@ -286,13 +287,12 @@ int llattn_num_levels(int T) {
 
 llattn_status llattn_workspace_bytes(int in_dtype, int path, int chunk, int B, int H, int T,
                                      int dk, int dv, int varlen, size_t* bytes) {
-  (void)varlen;  // dense and packed batches are sized alike (T bounds every sequence)
   if (!bytes) return LLATTN_ERR_ARG;
   if (B < 0 || H < 0 || T < 0 || T > (1 << 24)) return LLATTN_ERR_SHAPE;
   if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
   llattn_status s = resolve(in_dtype, &path, &chunk, T, dk, dv);
   if (s != LLATTN_OK) return s;
-  *bytes = (B == 0 || H == 0 || T == 0) ? 0 : workspace_for(path, chunk, B, H, T, dk, dv);
+  *bytes = (B == 0 || H == 0 || T == 0) ? 0 : workspace_for(path, chunk, B, H, T, dk, dv, varlen != 0);
   return LLATTN_OK;
 }
 
@@ -360,6 +360,69 @@ llattn_status llattn_device_status(unsigned int* flags, int clear) {
   }
   *flags = v;
   return (v & LLATTN_DEV_WAIT_TIMEOUT) ? LLATTN_ERR_TIMEOUT : LLATTN_OK;
+}
+
+llattn_status llattn_gdn_fwd(int in_dtype, const void* q, const void* k, const void* v,
+                            const float* log_alpha, const float* beta, const float* lam,
+                            float* out, int B, int H, int T, int dk, int dv,
+                            const int* cu_seqlens, void* stream) {
+  if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+  if (B < 0 || H < 0 || T < 0 || H > 65535 || B > 65535) return LLATTN_ERR_SHAPE;
+  if (!head_dim_ok(dk) || !head_dim_ok(dv) || !llattn::gdn_supports(dk, dv, T))
+    return LLATTN_ERR_SHAPE;
+  if (B == 0 || H == 0 || T == 0) return LLATTN_OK;
+  if (!q || !k || !v || !log_alpha || !beta || !lam || !out) return LLATTN_ERR_ARG;
+  if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4) ||
+      !aligned(log_alpha, 4) || !aligned(beta, 4) || !aligned(lam, 4) ||
+      (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return LLATTN_ERR_ALIGN;
+  const void* ins[6] = {q, k, v, log_alpha, beta, lam};
+  for (const void* p : ins)
+    if (p == static_cast<const void*>(out)) return LLATTN_ERR_ARG;
+  const int L = llattn_num_levels(T);
+  if (cu_seqlens == nullptr) {
+    const unsigned long long ntok = (unsigned long long)B * T;
+    if (ntok * H * (unsigned long long)(dk > dv ? dk : dv) > (1ull << 40)) return LLATTN_ERR_SHAPE;
+    const size_t esz = in_dtype == LLATTN_BF16 ? 2 : 4;
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out);
+    const uintptr_t o1 = o0 + ntok * H * dv * sizeof(float);
+    const struct { const void* p; size_t n; } rng[6] = {
+        {q, ntok * H * dk * esz}, {k, ntok * H * dk * esz}, {v, ntok * H * dv * esz},
+        {log_alpha, ntok * H * sizeof(float)}, {beta, ntok * H * sizeof(float)},
+        {lam, ntok * H * L * sizeof(float)}};
+    for (const auto& r : rng) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(r.p), a1 = a0 + r.n;
+      if (a0 < o1 && o0 < a1) return LLATTN_ERR_ARG;
+    }
+  }
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  llattn_status s = device_state(&ds, &dev);
+  if (s != LLATTN_OK) return s;
+  llattn::GdnProblem p{in_dtype, q, k, v, log_alpha, beta, lam, out, B, H, T, dk, dv, L,
+                       cu_seqlens, ds->status};
+  const cudaError_t e = llattn::gdn_forward(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_set_segment_chunks(int chunks) {
+  if (chunks < 0 || chunks > (1 << 20) || (chunks > 0 && !pow2(chunks)) || chunks == 1)
+    return LLATTN_ERR_ARG;
+  llattn::tc_set_segment_chunks(chunks);
+  return LLATTN_OK;
+}
+
+llattn_status llattn_segment_plan(int B, int H, int T, int dk, int dv, int varlen,
+                                  int* chunks_per_segment) {
+  if (!chunks_per_segment) return LLATTN_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || T > (1 << 24)) return LLATTN_ERR_SHAPE;
+  if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
+  *chunks_per_segment = 0;
+  if (B == 0 || H == 0 || T == 0 || !llattn::tc_supports(LLATTN_BF16, dk, dv, 128, T))
+    return LLATTN_OK;
+  *chunks_per_segment = llattn::tc_segment_chunks(B, H, T, dk, dv, varlen != 0);
+  return LLATTN_OK;
 }
 
 llattn_status llattn_stream_status(unsigned int* flags, int clear, void* stream) {

@@ -30,12 +30,16 @@ void main_kernel_end(cudaStream_t st);
 
 // Bytes of scratch each path needs (256-byte granules).
 size_t simt_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk);
-size_t tc_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk);
+size_t tc_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk, bool varlen);
 
 // Kernel launchers; return a cudaError_t from the launches.
 cudaError_t simt_forward(const Problem& p, int chunk, void* ws, cudaStream_t st);
 cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, bool serial);
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T);
+// Segment length of the tensor-core path: the forced value (chunks, 0 = automatic), and the
+// chunks per segment a call of this shape uses (0: each CTA walks a whole sequence).
+void tc_set_segment_chunks(int chunks);
+int tc_segment_chunks(int nseq, int H, int T, int dk, int dv, bool varlen);
 bool tc_serial_supports(int in_dtype, int dk, int dv, int chunk, int T);
 
 // Device address of the fixed scratch array behind llattn_fwd_noalloc on the

@@ -545,7 +545,7 @@ constexpr int kPI2 = 18;                      // warp of the inter-chunk MMA iss
 
 constexpr int kPG = 3;                        // g buffers
 constexpr uint32_t kPLamStride = 9;           // group A lam table: levels 0..7, odd stride
-constexpr int kPNumBars = 30;
+constexpr int kPNumBars = 31;
 
 // Shared-memory map of the pipelined kernel for NLEV chunk-level Fenwick states kept on chip
 // (T <= 128 * 2^NLEV) and an NST-stage Q/K/V ring (chunk c in stage c % NST).
@@ -568,6 +568,7 @@ struct PipeLayout {
 };
 using PipeShort = PipeLayout<6, 3>;   // T <= 8192
 using PipeLong = PipeLayout<7, 2>;    // T <= 16384
+using PipeXL = PipeLayout<10, 2>;     // T <= 131072 (long sequences, walked in segments)
 
 constexpr uint32_t kPColSP = 0;    // S = Q K^T, overwritten in place by P (fp16)
 constexpr uint32_t kPColO = 128;   // P V accumulator
@@ -584,7 +585,7 @@ enum : int {
   B_FULL = 0, B_EMPTY = 3, B_SFULL = 6, B_PFULL = 7, B_SPEMPTY = 8, B_KS = 9, B_HFULL = 10,
   B_HEMPTY = 11, B_LV = 12, B_LV1 = 13, B_OFULL = 14, B_OEMPTY = 15, B_RFULL = 16,
   B_REMPTY = 17, B_GREADY = 18, B_GEMPTY = 21, B_DRAIN = 24, B_DRAIN2 = 25, B_OSTAGED = 26,
-  B_FREE = 29
+  B_FREE = 29, B_PREFILL = 30
 };
 
 // Wait on an mbarrier phase; returns false at once if the CTA has aborted, and aborts
@@ -631,11 +632,36 @@ __device__ __forceinline__ bool next_chain(int c, int from, int& b0, int& b1) {
   return true;
 }
 
+// Launch arguments of the pipelined kernel beyond the tensors.
+//   g          a CTA walks one segment of 2^g chunks (blockIdx.z); g >= 30: the whole sequence
+//   ndv        64-column tiles of v and out per head (blockIdx.x = head * ndv + tile)
+//   qcol       first q / k column this launch reads (d_k is taken 64 columns per launch)
+//   dk_tot, dv_tot   row lengths of q / k and of v / out
+//   accumulate add this launch's share into out (a later d_k slice) instead of storing it
+//   blocks, block_decay, nblk, nseg   the pre-filled levels: per (sequence, head tile),
+//              nblk dyadic block states over segments (fp16 slot images of 8 KB) and their
+//              total log decays; nseg = segments per sequence (the grid's z extent)
+struct SegArgs {
+  int g, ndv, qcol, dk_tot, dv_tot, accumulate;
+  const uint8_t* blocks;
+  const float* block_decay;
+  int nblk, nseg;
+};
+
+// Index of dyadic block (b, j) over segments (level b, even j: segments j*2^b .. (j+2)*2^b - 1
+// minus the upper half, i.e. the 2^b segments just before an odd multiple of 2^b) among the
+// blocks kept per (sequence, head tile): level b holds blocks_at_level(nseg, b) of them.
+__host__ __device__ inline int seg_block_index(int nseg, int b, int j) {
+  return level_offset(nseg, b) + (j >> 1);
+}
+
 // MN-major descriptor whose second 64-row group along M repeats the first (LBO = 0):
 // an M = 128 MMA over a 64-wide operand yields the 64-row result twice.
 __device__ __forceinline__ uint64_t mndesc_dup(uint32_t saddr) { return sdesc_sw128(saddr, 0, 1024); }
 
-template <int NLEV, int NST>
+// GEN = false: a whole (sequence, head) per CTA with d_k = d_v = 64; true: segments, 64-column
+// slices of wider heads and the accumulating pass (the SegArgs), at a few registers' cost.
+template <int NLEV, int NST, bool GEN>
 __global__ void __maxnreg__(96)
 tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
             const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
@@ -643,7 +669,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
             const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
             const float* __restrict__ log_a, const float* __restrict__ lam,
             float* __restrict__ out, int H, int T, int L, const int* __restrict__ cu,
-            unsigned int* status) {
+            unsigned int* status, const SegArgs sa) {
   using LY = PipeLayout<NLEV, NST>;
   constexpr int kLevels = NLEV;   // chunk-level states on chip in this instantiation
   constexpr int kPStages = NST;   // Q/K/V ring stages
@@ -655,11 +681,26 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   const int sub = warp & 3;
   const int row = sub * 32 + lane;
   const uint32_t lane_off = uint32_t(sub * 32) << 16;
-  const int h = blockIdx.x, sq = blockIdx.y;
+  // blockIdx.x = head * ndv + value tile (64 columns of v and out); blockIdx.z = segment
+  const int ndv = GEN ? sa.ndv : 1;
+  const int h = blockIdx.x / ndv, sq = blockIdx.y;
+  const int vcol = GEN ? (blockIdx.x % ndv) * kD : 0;   // first v / out column of this CTA
+  const int qcol = GEN ? sa.qcol : 0;                   // first q / k column of this launch
+  const int dk_tot = GEN ? sa.dk_tot : kD, dv_tot = GEN ? sa.dv_tot : kD;
+  const bool accum = GEN && sa.accumulate;
+  const int segg = GEN ? sa.g : 30;
 
   const SeqSpan sp = seq_span(sq, T, cu, status);
   if (sp.len <= 0) return;
-  const int nch = (sp.len + kC - 1) / kC;
+  // This CTA walks segment J: chunks c0 .. c0 + nch - 1 of the sequence, c0 = J * 2^g.
+  // Loops below run over the local index c (ring stages and barrier phases); the global
+  // chunk index c0 + c gives token positions and the Fenwick bits.  Levels g and above of
+  // the segment's chunks are the bits of J: their block states come pre-filled.
+  const int nch_seq = (sp.len + kC - 1) / kC;
+  const int J = blockIdx.z;
+  const int c0 = segg >= 30 ? 0 : (J << segg);
+  if (segg >= 30 ? J > 0 : c0 >= nch_seq) return;
+  const int nch = segg >= 30 ? nch_seq : min(nch_seq - c0, 1 << segg);
 
   auto stage = [sm](int i) { return sm + i * kStage; };
   uint8_t* slots = sm + LY::kOffSlots;
@@ -682,6 +723,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       uint32_t cnt = 1;  // TMA / tcgen05.commit arrivals
       if (i >= B_EMPTY && i < B_EMPTY + kPStages) cnt = 2;  // both MMA issuers
       if (i == B_PFULL || i == B_KS || (i >= B_GREADY && i < B_GREADY + kPG)) cnt = kPNA;
+      if (i == B_PREFILL) cnt = 1 + kPNB;   // the producer's copies and group B's Q copy
       if (i == B_HEMPTY || i == B_LV || i == B_LV1 || i == B_OEMPTY || i == B_REMPTY ||
           (i >= B_GEMPTY && i < B_GEMPTY + kPG) || (i >= B_OSTAGED && i < B_OSTAGED + kPStages))
         cnt = kPNB;
@@ -698,7 +740,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = misc[0];
   auto W = [&](int b, uint32_t parity) { return pwait(&bars[b], parity, abort_flag, status); };
-  auto is_full = [&](int c) { return (c + 1) * kC <= sp.len; };
+  auto is_full = [&](int c) { return (c0 + c + 1) * kC <= sp.len; };
+  auto tok_of = [&](int c) { return sp.start + (long long)(c0 + c) * kC; };   // first token
+  auto nrows = [&](int c) { return min(kC, sp.len - (c0 + c) * kC); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -713,14 +757,34 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       auto store_out = [&](int cc) {
         if (!W(B_OSTAGED + cc % kPStages, (cc / kPStages) & 1)) return false;
         if (is_full(cc)) {
-          const int tok0 = static_cast<int>(sp.start + (long long)cc * kC);
-          tma_store_3d(&tmo, stage(cc % kPStages), 0, h, tok0);
-          tma_store_3d(&tmo, stage(cc % kPStages) + kTile, 32, h, tok0);
+          const int tok0 = static_cast<int>(tok_of(cc));
+          if (accum) {   // a later d_k slice adds its share to the output
+            tma_reduce_add_3d(&tmo, stage(cc % kPStages), vcol, h, tok0);
+            tma_reduce_add_3d(&tmo, stage(cc % kPStages) + kTile, vcol + 32, h, tok0);
+          } else {
+            tma_store_3d(&tmo, stage(cc % kPStages), vcol, h, tok0);
+            tma_store_3d(&tmo, stage(cc % kPStages) + kTile, vcol + 32, h, tok0);
+          }
           bulk_commit();
           bulk_wait_read();
         }
         return true;
       };
+      if (c0 > 0) {
+        // block states of the levels above the segment (set bits of J), ahead of the loads
+        const uint8_t* blk = sa.blocks + (size_t)(sq * gridDim.x + blockIdx.x) * sa.nblk * 8192;
+        uint32_t bytes = 0;
+        for (int b = segg; b < NLEV; ++b)
+          if ((J >> (b - segg)) & 1) bytes += 8192;
+        mbar_arrive_expect_tx(&bars[B_PREFILL], bytes);
+        for (int b = segg; b < NLEV; ++b) {
+          const int bs = b - segg;
+          if ((J >> bs) & 1)
+            bulk_load(slots + b * 8192,
+                      blk + (size_t)seg_block_index(sa.nseg, bs, (J >> bs) - 1) * 8192, 8192,
+                      &bars[B_PREFILL]);
+        }
+      }
       for (int c = 0; c < nch; ++c) {
         const int s = c % kPStages, kk = c / kPStages;
         if (c >= kPStages && (!W(B_EMPTY + s, (kk & 1) ^ 1) || !store_out(c - kPStages))) {
@@ -728,11 +792,11 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
           break;
         }
         if (is_full(c)) {
-          const int tok0 = static_cast<int>(sp.start + (long long)c * kC);
+          const int tok0 = static_cast<int>(tok_of(c));
           mbar_arrive_expect_tx(&bars[B_FULL + s], 3 * kTile);
-          tma_load_3d(stage(s), &tmq, &bars[B_FULL + s], 0, h, tok0);
-          tma_load_3d(stage(s) + kTile, &tmk, &bars[B_FULL + s], 0, h, tok0);
-          tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[B_FULL + s], 0, h, tok0);
+          tma_load_3d(stage(s), &tmq, &bars[B_FULL + s], qcol, h, tok0);
+          tma_load_3d(stage(s) + kTile, &tmk, &bars[B_FULL + s], qcol, h, tok0);
+          tma_load_3d(stage(s) + 2 * kTile, &tmv, &bars[B_FULL + s], vcol, h, tok0);
           if (s == 0) last0 = c; else if (s == 1) last1 = c; else last2 = c;
         } else {
           mbar_arrive(&bars[B_FREE]);
@@ -742,6 +806,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       bulk_wait_all();  // output tiles written
       if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) {
         // an aborted CTA still lets its own copies land before it exits
+        if (c0 > 0) mbar_wait(&bars[B_PREFILL], 0, 200000000ull);
         if (last0 >= 0) mbar_wait(&bars[B_FULL + 0], (last0 / kPStages) & 1, 200000000ull);
         if (last1 >= 0) mbar_wait(&bars[B_FULL + 1], (last1 / kPStages) & 1, 200000000ull);
         if (last2 >= 0) mbar_wait(&bars[B_FULL + 2], (last2 / kPStages) & 1, 200000000ull);
@@ -792,7 +857,8 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     float pf[kNP];
     float pf_la = 0.f;
     auto prefetch = [&](int c) {
-      const int t = c * kC + row;
+      const int cg = c0 + c;
+      const int t = cg * kC + row;
       const bool okt = t < sp.len;
       const long long tok = sp.start + t;
       const float* lr = lam + (tok * H + h) * L;
@@ -801,7 +867,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         const int l = part + 2 * i;
         // inter-chunk levels only where chunk c reads them (bit l - 1 - log2 C of c): each
         // row load that touches another cache sector costs the mask/scan warps time
-        const bool need = l <= kLogC || ((c >> (l - 1 - kLogC)) & 1);
+        const bool need = l <= kLogC || ((cg >> (l - 1 - kLogC)) & 1);
         pf[i] = (okt && l < L && need) ? __ldg(lr + l) : 0.f;
       }
       if (part == 0) pf_la = okt ? __ldg(log_a + tok * H + h) : 0.f;
@@ -819,7 +885,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     // bulk copies holds; it is a hint and changes no result.
     auto l2_prefetch = [&](int cc) {
       if (cc >= nch || !is_full(cc)) return;
-      const long long tok0 = sp.start + (long long)cc * kC;
+      const long long tok0 = tok_of(cc);
       const float* lb = lam + (tok0 * H + (long long)h * kC) * L;    // share h of the block
       const float* ab = log_a + tok0 * H + (long long)h * kC;
       if (((reinterpret_cast<uintptr_t>(lb) | (uint32_t)(kC * L * 4)) & 15u) == 0)
@@ -829,7 +895,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     auto decay_scan = [&](int c) {
       const int gb = c % kPG, gk = c / kPG;  // g buffer and its use index
       if (wa == 0 && lane == 0) l2_prefetch(c + 2);
-      const int n = min(kC, sp.len - c * kC);
+      const int n = nrows(c);
       float pfc[kNP];
 #pragma unroll
       for (int i = 0; i < kNP; ++i) pfc[i] = pf[i];
@@ -877,21 +943,23 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     decay_scan(0);
     for (int c = 0; c < nch; ++c) {
       const int s = c % kPStages, kk = c / kPStages;
-      const int n = min(kC, sp.len - c * kC);
+      const int n = nrows(c);
       if (!is_full(c)) {
         // ragged last chunk: plain loads into the stage, rows past the end zero-filled, once
         // the producer has stored the output tile of chunk c - 3 from it
         W(B_FREE, 0);
-        const long long tok0 = sp.start + (long long)c * kC;
+        const long long tok0 = tok_of(c);
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
           const __nv_bfloat16* src = tsr == 0 ? q : (tsr == 1 ? k : v);
+          const int rowlen = tsr == 2 ? dv_tot : dk_tot;
+          const int col0 = tsr == 2 ? vcol : qcol;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int col = part * 32 + j * 8;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
             if (row < n) {
-              val = *reinterpret_cast<const uint4*>(src + ((tok0 + row) * H + h) * kD + col);
+              val = *reinterpret_cast<const uint4*>(src + ((tok0 + row) * H + h) * rowlen + col0 + col);
               if (tsr == 2) val = bf16x8_to_f16x8(val);   // V in fp16
             }
             *reinterpret_cast<uint4*>(stage(s) + tsr * kTile + sw128_off(row, col)) = val;
@@ -1012,13 +1080,37 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     float gtot[kLevels];
 #pragma unroll
     for (int b = 0; b < kLevels; ++b) gtot[b] = 0.f;
+    if (c0 > 0) {
+      // The first chunk of a later segment reads the levels above the segment: its fp16 Q
+      // copy (made for every other chunk during the previous merge) is made here, and the
+      // pre-fill barrier, which the readouts wait for, also waits for it.
+      W(B_FULL, 0);
+      {
+        const uint4* qsrc = reinterpret_cast<const uint4*>(stage(0));
+        uint4* qdst = reinterpret_cast<uint4*>(qh);
+        const int t = (warp - kPB0) * 32 + lane;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qdst[t + 256 * i] = bf16x8_to_f16x8(qsrc[t + 256 * i]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_PREFILL]);
+      // total log decay of each pre-filled block (levels g.. : the set bits of J)
+      const float* bd = sa.block_decay + (size_t)(sq * gridDim.x + blockIdx.x) * sa.nblk;
+#pragma unroll
+      for (int b = 0; b < kLevels; ++b) {
+        const int bs = b - segg;
+        if (bs >= 0 && ((J >> bs) & 1)) gtot[b] = bd[seg_block_index(sa.nseg, bs, (J >> bs) - 1)];
+      }
+    }
     uint32_t u = 0;
     // An fp16 operand out of range (|x| >= 65520 rounds to inf) reaches the output as inf
-    // or NaN, so checking every output value catches it; the host sees a status bit.
-    bool nonfinite = false;
+    // or NaN.  Any such value makes this thread's running sum of its outputs inf or NaN, so
+    // one check of the sum at the end catches it; the host sees a status bit.
+    float osum = 0.f;
     for (int c = 0; c < nch; ++c) {
       const int s = c % kPStages;
-      const int n = min(kC, sp.len - c * kC);
+      const int n = nrows(c);
+      const int cg = c0 + c;   // global chunk index: its bits are the levels read
       W(B_GREADY + c % kPG, (c / kPG) & 1);
       const float gend = gs[(c % kPG) * kC + n - 1];
       const float* lamv = lamB + ((c % kPG) * kC + row) * kLevels;
@@ -1041,14 +1133,14 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       int cur0 = -1, cur1 = -1;  // readout chain being drained
 #pragma unroll
       for (int b = 0; b < kLevels; ++b) {
-        if (!((c >> b) & 1)) continue;
+        if (!((cg >> b) & 1)) continue;
         if (b > cur1) {
           if (cur1 >= 0) {
             tc_fence_before();
             mbar_arrive(&bars[B_REMPTY]);
             ++u;
           }
-          next_chain<NLEV>(c, b, cur0, cur1);
+          next_chain<NLEV>(cg, b, cur0, cur1);
           W(B_RFULL, u & 1);
           tc_fence_after();
         }
@@ -1068,7 +1160,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
       // ---- Fenwick merge: level m = H + sum_{b<m} exp(decay after block b) S_b ----
       if (c + 1 < nch) {
-        const int m = __ffs(~c) - 1;
+        const int m = __ffs(~cg) - 1;   // below g: a segment skips the merge after its last chunk
         // the lower levels do not depend on this chunk: sum them before H arrives
         float2 hv[8];
 #pragma unroll
@@ -1134,8 +1226,7 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
       }
       if (row < n) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          nonfinite |= !(fabsf(o2[e].x) <= 3.402823466e38f) | !(fabsf(o2[e].y) <= 3.402823466e38f);
+        for (int e = 0; e < 16; ++e) osum += o2[e].x + o2[e].y;
       }
       if (n == kC) {
         // Whole chunk: stage the 128 x 64 fp32 tile in the Q (columns 0..31) and K (32..63)
@@ -1151,16 +1242,25 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
         mbar_arrive(&bars[B_OSTAGED + s]);  // the producer stores the tile
       } else {
         if (row < n) {
-          float* dst = out + ((sp.start + (long long)c * kC + row) * H + h) * kD + 32 * half;
+          float* dst = out + ((tok_of(c) + row) * H + h) * dv_tot + vcol + 32 * half;
+          if (accum) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 2)
-            *reinterpret_cast<float4*>(dst + 2 * e) =
-                make_float4(o2[e].x, o2[e].y, o2[e + 1].x, o2[e + 1].y);
+            for (int e = 0; e < 16; ++e) {
+              atomicAdd(dst + 2 * e, o2[e].x);
+              atomicAdd(dst + 2 * e + 1, o2[e].y);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; e += 2)
+              *reinterpret_cast<float4*>(dst + 2 * e) =
+                  make_float4(o2[e].x, o2[e].y, o2[e + 1].x, o2[e + 1].y);
+          }
         }
         mbar_arrive(&bars[B_OSTAGED + s]);  // nothing staged; keeps the phases in step
       }
       mbar_arrive(&bars[B_GEMPTY + c % kPG]);
     }
+    const bool nonfinite = !(fabsf(osum) <= 3.402823466e38f);
     if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(status, LLATTN_DEV_NONFINITE);
   } else {
     // ------------------------------------------------------------ inter-chunk MMA issuer
@@ -1170,13 +1270,22 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
     // waiter, and a waiting issuer takes no issue slots from the math warps.
     if (lane == 0) {
       uint32_t u = 0;  // readout chains issued so far
+      bool prefilled = c0 == 0;
       for (int c = 0; c < nch; ++c) {
         const int s = c % kPStages;
         if (!W(B_FULL + s, (c / kPStages) & 1)) break;
         const uint32_t qa = smem_u32(stage(s)), ka = qa + kTile, va = qa + 2 * kTile;
         bool ok = true;
         int cb0 = 0, cb1 = 0;
-        for (bool more = next_chain<NLEV>(c, 0, cb0, cb1); more; more = next_chain<NLEV>(c, cb1 + 1, cb0, cb1)) {
+        const int cg = c0 + c;
+        for (bool more = next_chain<NLEV>(cg, 0, cb0, cb1); more; more = next_chain<NLEV>(cg, cb1 + 1, cb0, cb1)) {
+          if (!prefilled) {   // the block states above the segment have landed
+            if (!W(B_PREFILL, 0)) {
+              ok = false;
+              break;
+            }
+            prefilled = true;
+          }
           if ((c > 0 && !W(((c - 1) & 1) ? B_LV1 : B_LV, ((c - 1) >> 1) & 1)) ||
               !W(B_REMPTY, (u & 1) ^ 1)) {
             ok = false;
@@ -1217,6 +1326,248 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   }
 }
 
+// ==========================================================================================
+// Segment pre-pass.  A sequence walked in segments of 2^g chunks (one CTA each) needs, at the
+// start of segment J, the levels above the segment: for every set bit b of J, the state of the
+// 2^b segments just before J's aligned group of 2^(b+1) segments, decayed to that block's end.
+// That is the Fenwick binary counter of the walk kernel one level up, over segments instead
+// of chunks ([IT] "Partizionamento Gerarchico": the buckets are dyadic blocks, so a block of
+// segments is a union of whole lower blocks).  tc_seg_total computes each segment's total
+// state on the tensor cores; seg_blocks runs the counter and stores each block once, as the
+// fp16 slot image the walk kernel copies into shared memory.
+// ==========================================================================================
+constexpr int kSegThreads = 288;   // warp 0: TMA producer and MMA issuer (lane 0); warps 1..8: math
+constexpr int kSegMath = 256;
+constexpr uint32_t kSegSmem = 2 * 2 * kTile + kC * 4 + 64 + 64 + 1024;
+
+// One CTA per (head tile, sequence, segment J) for every segment but a sequence's last:
+//   seg_state[item] = sum over the segment's tokens s of exp(G_end - g_s) v_s k_s^T, stored
+//   [d_v][d_k] fp32 (the transposed state, as the walk kernel's merge forms it), and
+//   seg_decay[item] = the segment's total log decay G_end - G_start.
+// Chunks are taken last to first, so a running decay D (from the end of the chunk being
+// scaled to the end of the segment) folds into each token's factor and one TMEM accumulator
+// collects the whole sum: K~ = exp(D + sum_{r > s in chunk} log a_r) K, fp16, factors <= 1.
+__global__ void __launch_bounds__(kSegThreads, 1)
+tc_seg_total(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+             const float* __restrict__ log_a, int H, int T, const int* __restrict__ cu,
+             unsigned int* status, const SegArgs sa, float* __restrict__ seg_state,
+             float* __restrict__ seg_decay) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x / sa.ndv, sq = blockIdx.y, J = blockIdx.z;
+  const int vcol = (blockIdx.x % sa.ndv) * kD;
+  const SeqSpan sp = seq_span(sq, T, cu, status);
+  const int nch_seq = (sp.len + kC - 1) / kC;
+  const int c0 = J << sa.g;
+  // only segments followed by another one are read (and those are whole)
+  if (c0 + (1 << sa.g) >= nch_seq) return;
+  const int n = 1 << sa.g;
+  auto stage = [sm](int i) { return sm + i * 2 * kTile; };   // K tile, then V tile
+  float* fac = reinterpret_cast<float*>(sm + 4 * kTile);
+  float* part = fac + kC;                                     // scan carries (4 floats)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 4 * kTile + kC * 4 + 64);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 6);     // [0] TMEM base, [1] abort
+  uint32_t* abort_flag = &misc[1];
+  enum { S_FULL = 0, S_SCALED = 2, S_MDONE = 3, S_DRAIN = 4 };
+  if (warp == 0) {
+    tmem_alloc(&misc[0], 64);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&bars[S_FULL], 1);
+    mbar_init(&bars[S_FULL + 1], 1);
+    mbar_init(&bars[S_SCALED], kSegMath);
+    mbar_init(&bars[S_MDONE], 1);
+    mbar_init(&bars[S_DRAIN], 1);
+    fence_mbar_init();
+    misc[1] = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  auto W = [&](int b, uint32_t parity) { return pwait(&bars[b], parity, abort_flag, status); };
+  // chunk processed at step i (last chunk first)
+  auto chunk_tok = [&](int i) { return sp.start + (long long)(c0 + n - 1 - i) * kC; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      auto load = [&](int i) {
+        const int s = i & 1;
+        const int tok0 = static_cast<int>(chunk_tok(i));
+        mbar_arrive_expect_tx(&bars[S_FULL + s], 2 * kTile);
+        tma_load_3d(stage(s), &tmk, &bars[S_FULL + s], sa.qcol, h, tok0);
+        tma_load_3d(stage(s) + kTile, &tmv, &bars[S_FULL + s], vcol, h, tok0);
+      };
+      load(0);
+      if (n > 1) load(1);
+      int issued = 0, loads = n > 1 ? 2 : 1;
+      for (int i = 0; i < n; ++i) {
+        if (!W(S_SCALED, i & 1)) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(stage(i & 1)), va = ka + kTile;
+        const uint64_t vd = mndesc_dup(va), kd = mndesc(ka);
+#pragma unroll
+        for (int x = 0; x < kC / 16; ++x)
+          mma_ss(tmem, vd + 128 * x, kd + 128 * x, kIdescHT, (i > 0 || x > 0) ? 1u : 0u);
+        mma_commit(&bars[S_MDONE]);
+        ++issued;
+        if (i + 2 < n) {   // the stage is free once this chunk's MMAs are done
+          if (!W(S_MDONE, i & 1)) break;
+          load(i + 2);
+          ++loads;
+        }
+      }
+      mma_commit(&bars[S_DRAIN]);
+      mbar_wait(&bars[S_DRAIN], 0, 200000000ull);
+      if (*reinterpret_cast<volatile uint32_t*>(abort_flag)) {
+        // let this CTA's loads land before it exits
+        for (int i = (loads > 2 ? loads - 2 : 0); i < loads; ++i)
+          mbar_wait(&bars[S_FULL + (i & 1)], (i >> 1) & 1, 200000000ull);
+      }
+      (void)issued;
+    }
+  } else {
+    // ------------------------------------------------ math warps: factors, K~ and V in fp16
+    const int t = tid - 32;            // 0..255
+    const int w = t >> 5;              // 0..7
+    float D = 0.f;                     // log decay from the current chunk's end to the segment end
+    // (a failed wait does not leave the loop: the named barriers below stay matched, and an
+    // aborted CTA writes nothing)
+    for (int i = 0; i < n; ++i) {
+      const int s = i & 1;
+      W(S_FULL + s, (i >> 1) & 1);
+      // inclusive prefix of log a inside the chunk by the first four warps
+      float x = 0.f;
+      if (t < kC) {
+        x = __ldg(log_a + (chunk_tok(i) + t) * H + h);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) part[w] = x;
+      }
+      named_sync(1, kSegMath);
+      const float Gc = part[0] + part[1] + part[2] + part[3];
+      if (t < kC) {
+        float off = 0.f;
+        for (int q2 = 0; q2 < w; ++q2) off += part[q2];
+        fac[t] = __expf(D + Gc - (x + off));   // exp(D + sum of log a after token t)
+      }
+      named_sync(1, kSegMath);
+      // K rows scaled by their factor, V converted, both to fp16 in place
+      uint8_t* kt = stage(s);
+      uint4* vt = reinterpret_cast<uint4*>(stage(s) + kTile);
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int unit = t + kSegMath * u4;            // 16-byte unit of the 128 x 128 B tile
+        const float f = fac[unit >> 3];
+        uint4 raw = *reinterpret_cast<const uint4*>(kt + unit * 16);
+        uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+          wv[e] = pack_f16(pr.x * f, pr.y * f);
+        }
+        *reinterpret_cast<uint4*>(kt + unit * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        vt[unit] = bf16x8_to_f16x8(vt[unit]);
+      }
+      fence_proxy_async_smem();
+      D += Gc;
+      // one phase of S_SCALED at a time: the issuer has seen the previous one once its MMAs
+      // of the previous chunk are done
+      if (i > 0) W(S_MDONE, (i - 1) & 1);
+      mbar_arrive(&bars[S_SCALED]);
+    }
+    if (W(S_MDONE, (n - 1) & 1) && !*reinterpret_cast<volatile uint32_t*>(abort_flag)) {
+      tc_fence_after();
+      // H^T rows (d_v) sit in TMEM lanes 0..63; warps with w % 4 in {0, 1} read them
+      const int wq = (tid >> 5) & 3;
+      if (wq < 2) {
+        const int half = (tid >> 5) >= 5 ? 1 : 0;      // warps 1, 4 -> columns 0..31; 5, 8 -> 32..63
+        float r[32];
+        tmem_ld32(tmem + (uint32_t(wq * 32) << 16) + 32 * half, r);
+        tmem_wait_ld();
+        const size_t item = ((size_t)sq * gridDim.x + blockIdx.x) * (sa.nseg - 1) + J;
+        float* dst = seg_state + item * (kD * kD) + (wq * 32 + lane) * kD + 32 * half;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+        if (t == 0) seg_decay[item] = D;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// One CTA per (head tile, sequence): the binary counter over the sequence's segments.  After
+// segment J's total is merged, the block it completes - the 2^m segments ending at J, m the
+// trailing ones of J - is stored as an fp16 slot image ([d_v][d_k], 128-byte swizzle, the
+// layout of the walk kernel's level states) with its total log decay.  Each thread owns 16
+// consecutive elements of every state, so no thread reads another's.
+constexpr int kBlkThreads = 256;
+__global__ void __launch_bounds__(kBlkThreads)
+seg_blocks(int T, const int* __restrict__ cu, unsigned int* status, const SegArgs sa,
+           const float* __restrict__ seg_state, const float* __restrict__ seg_decay,
+           uint8_t* __restrict__ blocks, float* __restrict__ block_decay) {
+  extern __shared__ float cnt[];   // [levels][4096] fp32: the counter's slots
+  const int t = threadIdx.x, sq = blockIdx.y;
+  const SeqSpan sp = seq_span(sq, T, cu, status);
+  const int nch_seq = (sp.len + kC - 1) / kC;
+  const int nsq = (nch_seq + (1 << sa.g) - 1) >> sa.g;   // this sequence's segments
+  const size_t pair = (size_t)sq * gridDim.x + blockIdx.x;
+  const int r = t >> 2, col0 = (t & 3) * 16;             // this thread: row r, columns col0..+15
+  float gdec[8];
+#pragma unroll
+  for (int b = 0; b < 8; ++b) gdec[b] = 0.f;
+  for (int J = 0; J + 1 < nsq; ++J) {
+    const size_t item = pair * (sa.nseg - 1) + J;
+    const float4* src = reinterpret_cast<const float4*>(seg_state + item * (kD * kD) + r * kD + col0);
+    float x[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const float4 f = src[q4];
+      x[4 * q4] = f.x; x[4 * q4 + 1] = f.y; x[4 * q4 + 2] = f.z; x[4 * q4 + 3] = f.w;
+    }
+    const int m = __ffs(~J) - 1;
+    float acc = seg_decay[item];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (b < m) {
+        const float f = __expf(acc);
+        const float* sl = cnt + b * (kD * kD) + r * kD + col0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] += f * sl[e];
+        acc += gdec[b];
+      }
+    }
+    float* dsl = cnt + m * (kD * kD) + r * kD + col0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dsl[e] = x[e];
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+      if (b == m) gdec[b] = acc;
+    // block (m, j) with j = (J + 1) / 2^m - 1, read by segments J + 1 .. J + 2^m
+    const int blk = seg_block_index(sa.nseg, m, ((J + 1) >> m) - 1);
+    uint8_t* img = blocks + (pair * sa.nblk + blk) * 8192;
+#pragma unroll
+    for (int q8 = 0; q8 < 2; ++q8) {
+      uint32_t hv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hv[e] = pack_f16(x[8 * q8 + 2 * e], x[8 * q8 + 2 * e + 1]);
+      *reinterpret_cast<uint4*>(img + sw128_off(r, col0 + 8 * q8)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    }
+    if (t == 0) block_decay[pair * sa.nblk + blk] = acc;
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -1238,12 +1589,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [tokens, H, 64] bf16 viewed as a 3-D tensor {64, H, tokens}; box {64, 1, 128}, 128 B swizzle.
-cudaError_t make_map(CUtensorMap* m, const void* base, int H, long long tokens) {
+// [tokens, H, rowlen] bf16 viewed as a 3-D tensor {rowlen, H, tokens}; box {64, 1, 128}
+// (one 64-column slice of a row), 128 B swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, int rowlen, int H, long long tokens) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t dims[3] = {kD, (cuuint64_t)H, (cuuint64_t)tokens};
-  const cuuint64_t strides[2] = {kD * 2, (cuuint64_t)H * kD * 2};
+  const cuuint64_t dims[3] = {(cuuint64_t)rowlen, (cuuint64_t)H, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)rowlen * 2, (cuuint64_t)H * rowlen * 2};
   const cuuint32_t box[3] = {kD, 1, kC};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
@@ -1252,12 +1604,12 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int H, long long tokens) 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// out [tokens, H, 64] fp32 as {64, H, tokens}; box {32, 1, 128} (128 B rows), 128 B swizzle.
-cudaError_t make_out_map(CUtensorMap* m, void* base, int H, long long tokens) {
+// out [tokens, H, rowlen] fp32 as {rowlen, H, tokens}; box {32, 1, 128} (128 B rows), 128 B swizzle.
+cudaError_t make_out_map(CUtensorMap* m, void* base, int rowlen, int H, long long tokens) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t dims[3] = {kD, (cuuint64_t)H, (cuuint64_t)tokens};
-  const cuuint64_t strides[2] = {kD * 4, (cuuint64_t)H * kD * 4};
+  const cuuint64_t dims[3] = {(cuuint64_t)rowlen, (cuuint64_t)H, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)rowlen * 4, (cuuint64_t)H * rowlen * 4};
   const cuuint32_t box[3] = {32, 1, kC};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
@@ -1266,22 +1618,130 @@ cudaError_t make_out_map(CUtensorMap* m, void* base, int H, long long tokens) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// How a call is cut into CTAs.  One CTA (one per SM: shared memory and TMEM) walks 2^g chunks
+// of one (sequence, head, 64-column value tile); a whole sequence when g = kNoSplit.  The time
+// estimate, in chunk steps, is waves x (2^g + 2 steps of pipeline fill), plus the pre-pass for
+// split sequences (about 2 steps of launches and a step per 8 chunk-tiles per SM of segment
+// totals).  Packed batches count items at half the length bound (T only bounds them).
+constexpr int kNoSplit = 30;
+struct SegPlan {
+  int g = kNoSplit, nseg = 1, nblk = 0;
+};
+
+std::atomic<int> g_seg_chunks_override{0};   // llattn_set_segment_chunks
+
+SegPlan seg_plan(int nseq, int H, int T, int dk, int dv, bool varlen) {
+  (void)dk;
+  SegPlan pl;
+  const int nch = (T + kC - 1) / kC;
+  const int forced = g_seg_chunks_override.load();
+  if (forced > 0) {
+    int g = 0;
+    while ((1 << g) < forced) ++g;
+    if ((1 << g) >= nch) return pl;   // one segment covers every sequence
+    const int nseg = (nch + (1 << g) - 1) >> g;
+    if (chunk_levels(nseg) <= 8) {
+      pl.g = g;
+      pl.nseg = nseg;
+      pl.nblk = total_blocks(nseg);
+      return pl;
+    }
+  }
+  const int vh = H * (dv / kD);
+  const int nsm = sm_count();
+  const double per = varlen ? 0.5 : 1.0;
+  auto waves = [&](long long items) { return (double)((items + nsm - 1) / nsm); };
+  double best = waves((long long)nseq * vh) * (nch + 2);
+  for (int g = 1; (1 << g) < nch; ++g) {
+    const int nseg = (nch + (1 << g) - 1) >> g;
+    if (chunk_levels(nseg) > 8) continue;   // the counter over segments keeps <= 8 levels
+    const long long items = (long long)nseq * vh * ((long long)(per * nch + (1 << g) - 1) >> g);
+    const double pre = 2.0 + (double)nseq * vh * (per * nch) / (8.0 * nsm);
+    const double est = waves(items) * ((1 << g) + 2) + pre;
+    if (est < best) {
+      best = est;
+      pl.g = g;
+      pl.nseg = nseg;
+    }
+  }
+  pl.nblk = pl.nseg > 1 ? total_blocks(pl.nseg) : 0;
+  return pl;
+}
+
+struct SegWorkspace {
+  float* seg_state = nullptr;
+  float* seg_decay = nullptr;
+  uint8_t* blocks = nullptr;
+  float* block_decay = nullptr;
+  size_t bytes = 0;
+};
+
+SegWorkspace seg_workspace(const SegPlan& pl, int nseq, int H, int dv, void* base) {
+  SegWorkspace w;
+  if (pl.nseg <= 1) return w;
+  const size_t pairs = (size_t)nseq * H * (dv / kD);
+  const size_t items = pairs * (pl.nseg - 1);
+  const size_t a = round_up(items * kD * kD * sizeof(float), 256);
+  const size_t b = round_up(items * sizeof(float), 256);
+  const size_t c = round_up(pairs * pl.nblk * 8192, 256);
+  const size_t d = round_up(pairs * pl.nblk * sizeof(float), 256);
+  w.bytes = a + b + c + d;
+  if (base != nullptr) {
+    uint8_t* p = static_cast<uint8_t*>(base);
+    w.seg_state = reinterpret_cast<float*>(p);
+    w.seg_decay = reinterpret_cast<float*>(p + a);
+    w.blocks = p + a + b;
+    w.block_decay = reinterpret_cast<float*>(p + a + b + c);
+  }
+  return w;
+}
+
+template <typename LY, bool GEN>
+void launch_walk(const dim3& grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
+                 const CUtensorMap& mv, const CUtensorMap& mo, const Problem& p,
+                 const SegArgs& sa) {
+  tc_fwd_pipe<LY::kLev, LY::kSt, GEN><<<grid, kPThreads, LY::kSmemBytes, st>>>(
+      mq, mk, mv, mo, static_cast<const __nv_bfloat16*>(p.q),
+      static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v), p.log_a,
+      p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens, p.status, sa);
+}
+
 }  // namespace
 
-// The pipelined kernel keeps up to 7 chunk-level states on chip (T <= 16384); the serial
-// cross-check keeps 6 (T <= 8192).
+// The pipelined kernel keeps one fp16 state per chunk level on chip: 6 levels for T <= 8192,
+// 7 for T <= 16384 and 10 for T <= 131072 (walked in segments with the levels above a
+// segment pre-filled).  d_k and d_v are 64 or 128: 64-column slices of q . k add up, and
+// value columns are independent.  The serial cross-check takes d = 64, T <= 8192.
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T) {
-  return in_dtype == LLATTN_BF16 && dk == kD && dv == kD && chunk == kC &&
-         T <= kC * (1 << PipeLong::kLev);
+  return in_dtype == LLATTN_BF16 && (dk == 64 || dk == 128) && (dv == 64 || dv == 128) &&
+         chunk == kC && T <= kC * (1 << PipeXL::kLev);
 }
 
 bool tc_serial_supports(int in_dtype, int dk, int dv, int chunk, int T) {
-  return tc_supports(in_dtype, dk, dv, chunk, T) && T <= kC * kMaxChunks;
+  return in_dtype == LLATTN_BF16 && dk == kD && dv == kD && chunk == kC && T <= kC * kMaxChunks;
 }
 
-size_t tc_workspace_bytes(int, int, int, int, int, int) { return 0; }
+void tc_set_segment_chunks(int chunks) { g_seg_chunks_override.store(chunks); }
 
-cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool serial) {
+int tc_segment_chunks(int nseq, int H, int T, int dk, int dv, bool varlen) {
+  const SegPlan pl = seg_plan(nseq, H, T, dk, dv, varlen);
+  return pl.nseg > 1 ? (1 << pl.g) : 0;
+}
+
+size_t tc_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk, bool varlen) {
+  (void)chunk;
+  return seg_workspace(seg_plan(nseq, H, T, dk, dv, varlen), nseq, H, dv, nullptr).bytes;
+}
+
+cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, bool serial) {
   if (!(serial ? tc_serial_supports : tc_supports)(p.in_dtype, p.dk, p.dv, chunk, p.T))
     return cudaErrorNotSupported;
   // TMA only ever fetches whole chunks inside a sequence, so the token extent can be
@@ -1290,11 +1750,11 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
   if (tokens >= (1ll << 31)) return cudaErrorNotSupported;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  if ((e = make_map(&mq, p.q, p.H, tokens)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, p.k, p.H, tokens)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, p.v, p.H, tokens)) != cudaSuccess) return e;
+  if ((e = make_map(&mq, p.q, p.dk, p.H, tokens)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, p.k, p.dk, p.H, tokens)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, p.v, p.dv, p.H, tokens)) != cudaSuccess) return e;
   CUtensorMap mo;
-  if ((e = make_out_map(&mo, p.out, p.H, tokens)) != cudaSuccess) return e;
+  if ((e = make_out_map(&mo, p.out, p.dv, p.H, tokens)) != cudaSuccess) return e;
   // the shared-memory opt-in is a per-device attribute of each kernel
   static std::atomic<bool> attr_set[64];
   int dev = 0;
@@ -1304,33 +1764,69 @@ cudaError_t tc_forward(const Problem& p, int chunk, void*, cudaStream_t st, bool
     if ((e = cudaFuncSetAttribute(tc_fwd_serial, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kSmemBytes)) != cudaSuccess)
       return e;
-    if ((e = cudaFuncSetAttribute(tc_fwd_pipe<PipeShort::kLev, PipeShort::kSt>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)PipeShort::kSmemBytes)) != cudaSuccess)
+    const struct { const void* fn; int bytes; } walks[5] = {
+        {(const void*)tc_fwd_pipe<PipeShort::kLev, PipeShort::kSt, false>, (int)PipeShort::kSmemBytes},
+        {(const void*)tc_fwd_pipe<PipeLong::kLev, PipeLong::kSt, false>, (int)PipeLong::kSmemBytes},
+        {(const void*)tc_fwd_pipe<PipeShort::kLev, PipeShort::kSt, true>, (int)PipeShort::kSmemBytes},
+        {(const void*)tc_fwd_pipe<PipeLong::kLev, PipeLong::kSt, true>, (int)PipeLong::kSmemBytes},
+        {(const void*)tc_fwd_pipe<PipeXL::kLev, PipeXL::kSt, true>, (int)PipeXL::kSmemBytes}};
+    for (const auto& f : walks)
+      if ((e = cudaFuncSetAttribute(f.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, f.bytes)) !=
+          cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(tc_seg_total, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kSegSmem)) != cudaSuccess)
       return e;
-    if ((e = cudaFuncSetAttribute(tc_fwd_pipe<PipeLong::kLev, PipeLong::kSt>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)PipeLong::kSmemBytes)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(seg_blocks, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  8 * kD * kD * (int)sizeof(float))) != cudaSuccess)
       return e;
     attr_set[dev].store(true);
   }
-  const dim3 grid(p.H, p.nseq);
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(p.k);
-  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(p.v);
   main_kernel_begin(st);
-  if (serial)
-    tc_fwd_serial<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, q, k, v, p.log_a, p.lam, p.out,
-                                                      p.H, p.T, p.L, p.cu_seqlens, p.status);
-  else if (p.T <= kC * (1 << PipeShort::kLev))   // 6 levels on chip, three-stage ring
-    tc_fwd_pipe<PipeShort::kLev, PipeShort::kSt><<<grid, kPThreads, PipeShort::kSmemBytes, st>>>(
-        mq, mk, mv, mo, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens, p.status);
-  else                                            // 7 levels, two stages (shared memory)
-    tc_fwd_pipe<PipeLong::kLev, PipeLong::kSt><<<grid, kPThreads, PipeLong::kSmemBytes, st>>>(
-        mq, mk, mv, mo, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens, p.status);
+  if (serial) {
+    const dim3 grid(p.H, p.nseq);
+    tc_fwd_serial<<<grid, kThreads, kSmemBytes, st>>>(
+        mq, mk, mv, static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+        static_cast<const __nv_bfloat16*>(p.v), p.log_a, p.lam, p.out, p.H, p.T, p.L,
+        p.cu_seqlens, p.status);
+    main_kernel_end(st);
+    count_launch();
+    return cudaGetLastError();
+  }
+  const bool varlen = p.cu_seqlens != nullptr;
+  const SegPlan pl = seg_plan(p.nseq, p.H, p.T, p.dk, p.dv, varlen);
+  const SegWorkspace w = seg_workspace(pl, p.nseq, p.H, p.dv, ws);
+  if (pl.nseg > 1 && ws == nullptr) return cudaErrorInvalidValue;
+  const int ndv = p.dv / kD, vh = p.H * ndv;
+  const int nch = (p.T + kC - 1) / kC;
+  // every d_k slice of 64 columns is one pass; the later ones add into out
+  for (int i = 0; i < p.dk / kD; ++i) {
+    const SegArgs sa{pl.g, ndv, i * kD, p.dk, p.dv, i > 0 ? 1 : 0, w.blocks, w.block_decay,
+                     pl.nblk, pl.nseg};
+    if (pl.nseg > 1) {
+      tc_seg_total<<<dim3(vh, p.nseq, pl.nseg - 1), kSegThreads, kSegSmem, st>>>(
+          mk, mv, p.log_a, p.H, p.T, p.cu_seqlens, p.status, sa, w.seg_state, w.seg_decay);
+      seg_blocks<<<dim3(vh, p.nseq), kBlkThreads, chunk_levels(pl.nseg) * kD * kD * sizeof(float),
+                   st>>>(p.T, p.cu_seqlens, p.status, sa, w.seg_state, w.seg_decay, w.blocks,
+                         w.block_decay);
+      count_launch(2);
+    }
+    const dim3 grid(vh, p.nseq, pl.nseg);
+    const bool gen = pl.nseg > 1 || p.dk != kD || p.dv != kD;
+    if (nch <= (1 << PipeShort::kLev)) {      // 6 levels on chip, three-stage ring
+      if (gen) launch_walk<PipeShort, true>(grid, st, mq, mk, mv, mo, p, sa);
+      else launch_walk<PipeShort, false>(grid, st, mq, mk, mv, mo, p, sa);
+    } else if (nch <= (1 << PipeLong::kLev)) {   // 7 levels, two stages (shared memory)
+      if (gen) launch_walk<PipeLong, true>(grid, st, mq, mk, mv, mo, p, sa);
+      else launch_walk<PipeLong, false>(grid, st, mq, mk, mv, mo, p, sa);
+    } else {                                  // 10 levels, two stages, always in segments
+      launch_walk<PipeXL, true>(grid, st, mq, mk, mv, mo, p, sa);
+    }
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) break;
+  }
   main_kernel_end(st);
-  count_launch();
-  return cudaGetLastError();
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 }  // namespace llattn

@@ -79,11 +79,12 @@ enum { LLATTN_F32 = 0, LLATTN_BF16 = 1 };
 /* Kernel paths for llattn_fwd_ex.
  *   AUTO            tcgen05 path where one exists for the shape, else SIMT.
  *   SIMT            CUDA-core kernels (any dk, dv in {32,64,128}; fp32 or bf16 inputs).
- *   TCGEN05         tensor-core kernel, warp-specialised pipeline (bf16 inputs, d_k = d_v =
- *                   64, chunk 128, T <= 16384; the serial cross-check T <= 8192; it
- *                   rounds P, V, the decay-scaled K and the level states once to fp16, so
- *                   those intermediates must stay below 6.5e4 in magnitude - true for
- *                   L2-normalised q, k and moderate v, lam; use SIMT otherwise).
+ *   TCGEN05         tensor-core kernel, warp-specialised pipeline (bf16 inputs, d_k and
+ *                   d_v in {64, 128}, chunk 128, T <= 131072; the serial cross-check d = 64,
+ *                   T <= 8192; it rounds P, V, the decay-scaled K and the level states once
+ *                   to fp16, so those intermediates must stay below 6.5e4 in magnitude -
+ *                   true for L2-normalised q, k and moderate v, lam; a value out of range
+ *                   sets LLATTN_DEV_NONFINITE; use SIMT then).
  *   TCGEN05_SERIAL  the same arithmetic with one warp group walking each chunk's steps in
  *                   order (a slower cross-check of the pipelined kernel). */
 enum {
@@ -169,6 +170,30 @@ LLATTN_API llattn_status llattn_fwd_ex(int in_dtype, int path, int chunk, const 
  * current device.  Synchronises the device.  *flags receives LLATTN_DEV_* bits.
  */
 LLATTN_API llattn_status llattn_device_status(unsigned int* flags, int clear);
+
+/*
+ * Segments of the tensor-core path.  Each CTA walks a run of 128-token chunks of one
+ * (sequence, head, 64-column value tile), keeping one fp16 state per Fenwick level of the run
+ * on chip.  Long sequences, or batches with fewer such runs than the GPU has SMs, are cut into
+ * aligned segments of 2^g chunks walked in parallel.  The levels above a segment (its
+ * position's set bits, one level up) come from two pre-pass kernels: the segments' total
+ * states on the tensor cores, then the Fenwick binary counter over segments, whose dyadic
+ * block states the walk copies in ([IT] section 2, "Partizionamento Gerarchico"; Spanish
+ * section 2, "Algoritmo de Entrenamiento (Chunk-scan)": the chunk-level scan, applied over
+ * groups of chunks).  The scratch for those states is part of llattn_workspace_bytes().
+ *
+ * llattn_segment_plan - the chunks per segment a tensor-core call of this shape uses
+ *   (*chunks_per_segment = 0: every CTA walks a whole sequence, or the shape has no
+ *   tensor-core path).  varlen != 0 for packed batches (T then bounds the lengths).
+ * llattn_set_segment_chunks - force the segment length for later calls of this process:
+ *   chunks = 0 restores the automatic choice, else a power of two >= 2 (a length that would
+ *   need more than 8 counter levels over segments falls back to the automatic choice).  A
+ *   tuning and testing knob; the result does not depend on it beyond rounding.  Not
+ *   thread-safe with respect to calls already being planned on other threads.
+ */
+LLATTN_API llattn_status llattn_segment_plan(int B, int H, int T, int dk, int dv, int varlen,
+                                             int* chunks_per_segment);
+LLATTN_API llattn_status llattn_set_segment_chunks(int chunks);
 
 /*
  * llattn_stream_status - the same read, ordered on one stream instead of the whole
@@ -337,6 +362,33 @@ LLATTN_API llattn_status llattn_bwd(int in_dtype, const void* q, const void* k, 
                                     int B, int H, int T, int dk_dim, int dv_dim,
                                     const int* cu_seqlens, void* workspace,
                                     size_t workspace_bytes, void* stream);
+
+/*
+ * llattn_gdn_fwd - forward of Log-Linear Gated DeltaNet, the second variant of the pages
+ * (gist.science "Log-Linear Attention", Italian "Sommario tecnico" section 2,
+ * "Generalizzazione"; Spanish "Variantes Propuestas" item 2: the log-linear structure applied
+ * to the gated delta rule).  The pages print no formula for it; the operation computed is
+ *
+ *   o_t = sum_{s <= t} lam[t, l(t,s)] * beta_s * (q_t^T A_t A_{t-1} ... A_{s+1} k_s) * v_s,
+ *   A_r = alpha_r (I - beta_r k_r k_r^T),   alpha_r = exp(log_alpha[r]),
+ *
+ * with l(t, s) the Fenwick level of llattn_fwd: one gated-delta state per Fenwick level,
+ * every occupied level taking the transition A_t, the token's write beta_t k_t v_t^T opening
+ * level 0, levels weighted by lam and merged on promotion.  With lam == 1 it is plain Gated
+ * DeltaNet; with A_t = alpha_t I it is llattn_fwd's operation with v_s scaled by beta_s.
+ *   in_dtype   LLATTN_BF16 or LLATTN_F32 (type of q, k, v).  Arithmetic and the state are fp32
+ *              on CUDA cores (the recurrent form, token by token; one warp per value column).
+ *   q, k       [B, T, H, dk] (packed: [total, H, dk]); the delta rule expects unit-norm k.
+ *   v          [B, T, H, dv];  log_alpha, beta [B, T, H] fp32;  lam [B, T, H, L] fp32.
+ *   out        [B, T, H, dv] fp32, fully overwritten (rows outside [0, total) untouched).
+ *   dk, dv in {32, 64, 128}, T <= 65536; cu_seqlens as in llattn_fwd.
+ * Pointers 4-byte aligned; out must not overlap an input.  Asynchronous on `stream`; no
+ * scratch memory.  Errors as llattn_fwd.
+ */
+LLATTN_API llattn_status llattn_gdn_fwd(int in_dtype, const void* q, const void* k,
+                                        const void* v, const float* log_alpha, const float* beta,
+                                        const float* lam, float* out, int B, int H, int T, int dk,
+                                        int dv, const int* cu_seqlens, void* stream);
 
 /*
  * Launch accounting, for benchmarks.  llattn_profile(1) starts recording a pair

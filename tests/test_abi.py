@@ -80,25 +80,51 @@ def test_workspace_query():
 
 
 def test_tensor_core_path_limits():
-    """The pipelined tensor-core kernel takes T <= 16384 (seven chunk levels on chip), the serial
-    cross-check T <= 8192; beyond that AUTO falls back to the CUDA-core path (no CUDA call)."""
+    """The pipelined tensor-core kernel takes d_k, d_v in {64, 128} and T <= 131072 (ten chunk
+    levels on chip, long sequences walked in segments); the serial cross-check d = 64 and
+    T <= 8192.  Beyond that AUTO falls back to the CUDA-core path (no CUDA call)."""
     ws = binding.workspace_bytes
-    for T in (1, 8192, 8193, 16384):
+    for T in (1, 8192, 8193, 16384, 65536, 131072):
         ws(binding.BF16, "tcgen05", 0, 2, 4, T, 64, 64, False)
+    for dk, dv in ((128, 128), (64, 128), (128, 64)):
+        ws(binding.BF16, "tcgen05", 0, 1, 2, 4096, dk, dv, False)
     ws(binding.BF16, "tcgen05_serial", 0, 2, 4, 8192, 64, 64, False)
-    for path, T in (("tcgen05", 16385), ("tcgen05_serial", 8193)):
+    for path, T, d in (("tcgen05", 131073, 64), ("tcgen05_serial", 8193, 64),
+                       ("tcgen05_serial", 256, 128), ("tcgen05", 256, 32)):
         with pytest.raises(binding.LLAttnError) as e:
-            ws(binding.BF16, path, 0, 2, 4, T, 64, 64, False)
+            ws(binding.BF16, path, 0, 2, 4, T, d, d, False)
         assert e.value.status == 8   # LLATTN_ERR_UNSUPPORTED
-    for dk in (32, 128):             # the tensor-core kernel is built for d = 64
-        with pytest.raises(binding.LLAttnError):
-            ws(binding.BF16, "tcgen05", 0, 1, 1, 256, dk, dk, False)
     with pytest.raises(binding.LLAttnError):   # bf16 inputs only
         ws(binding.F32, "tcgen05", 0, 1, 1, 256, 64, 64, False)
     # AUTO resolves without error for every supported shape (CUDA-core fallback beyond the limit)
-    for T in (16384, 16385, 65536):
+    for T in (16384, 16385, 65536, 200000):
         ws(binding.BF16, "auto", 0, 1, 16, T, 64, 64, False)
     ws(binding.BF16, "auto", 0, 1, 16, 65536, 128, 128, False)
+
+
+def test_segment_plan_and_its_scratch():
+    """Shapes with fewer whole-sequence walks than SMs are cut into segments (and then need
+    scratch for the segment states); the benchmark's B=4, H=32, T=8192 shape is not."""
+    plan = binding.segment_plan
+    assert plan(4, 32, 8192, 64, 64) == 0
+    assert binding.workspace_bytes(binding.BF16, "tcgen05", 0, 4, 32, 8192, 64, 64, False) == 0
+    c = plan(1, 16, 65536, 128, 128)
+    assert c >= 2 and c & (c - 1) == 0 and c < 512
+    assert binding.workspace_bytes(binding.BF16, "tcgen05", 0, 1, 16, 65536, 128, 128, False) > 0
+    assert plan(8, 16, 16384, 64, 64, varlen=True) > 0
+    assert plan(1, 4, 100, 64, 64) == 0          # a single chunk is never cut
+    assert plan(1, 4, 256, 32, 32) == 0          # no tensor-core path for d = 32
+    try:
+        binding.set_segment_chunks(4)
+        assert plan(4, 32, 8192, 64, 64) == 4
+        assert plan(1, 1, 512, 64, 64) == 0      # 4 chunks: one segment holds the sequence
+        assert binding.workspace_bytes(binding.BF16, "tcgen05", 0, 4, 32, 8192, 64, 64, False) > 0
+    finally:
+        binding.set_segment_chunks(0)
+    assert plan(4, 32, 8192, 64, 64) == 0
+    for bad in (-1, 1, 3, 6):
+        with pytest.raises(binding.LLAttnError):
+            binding.set_segment_chunks(bad)
 
 
 def _decode(**kw):
@@ -178,3 +204,28 @@ def test_bwd_argument_errors_before_launch(kw, status):
 
 def test_bwd_empty_problems_are_no_ops():
     assert _bwd(B=0) == 0 and _bwd(H=0) == 0 and _bwd(T=0) == 0
+
+
+def _gdn(**kw):
+    a = dict(in_dtype=1, q=0x1000, k=0x2000, v=0x3000, log_alpha=0x4000, beta=0x4800,
+             lam=0x5000, out=0x6000, B=1, H=1, T=16, dk=64, dv=64, cu=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return binding.lib().llattn_gdn_fwd(a["in_dtype"], vp(a["q"]), vp(a["k"]), vp(a["v"]),
+                                        vp(a["log_alpha"]), vp(a["beta"]), vp(a["lam"]),
+                                        vp(a["out"]), a["B"], a["H"], a["T"], a["dk"], a["dv"],
+                                        vp(a["cu"]) if a["cu"] else None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48), 2), (dict(dv=256), 2), (dict(T=-1), 2), (dict(T=65537), 2),
+    (dict(in_dtype=3), 4), (dict(q=0x1002), 3), (dict(beta=0x4802), 3),
+    (dict(beta=0), 1), (dict(out=0x1000), 1), (dict(out=0x4800), 1),
+])
+def test_gdn_argument_errors_before_launch(kw, status):
+    assert _gdn(**kw) == status
+
+
+def test_gdn_empty_problems_are_no_ops():
+    assert _gdn(B=0) == 0 and _gdn(H=0) == 0 and _gdn(T=0) == 0
+

@@ -275,3 +275,74 @@ def test_fwd_bf16_alias_matches_fwd():
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
     assert binding.stream_status(clear=True) == 0
+
+
+# ------------------------------------------------------------------------------------------------
+# Segments: a CTA walks 2^g chunks, the levels above its segment pre-filled from the block
+# states the pre-pass builds (segment totals on the tensor cores, then the counter over segments)
+# ------------------------------------------------------------------------------------------------
+class _forced_segments:
+    def __init__(self, chunks):
+        self.chunks = chunks
+
+    def __enter__(self):
+        binding.set_segment_chunks(self.chunks)
+
+    def __exit__(self, *exc):
+        binding.set_segment_chunks(0)
+
+
+@pytest.mark.parametrize("chunks", [2, 4, 8, 32])
+@pytest.mark.parametrize("mode", ["zero", "slow", "dist"])
+def test_segments_forced_lengths(chunks, mode):
+    # 63 chunks with a ragged tail: segments of 2..32 chunks, up to five levels pre-filled
+    w = I.shrink(W["t8k_d64_bf16"], B=2, H=2, T=8000)
+    inp = I.make_inputs(w, seed=31, log_a_mode=mode)
+    ref = O.llattn_recurrent(inp)
+    with _forced_segments(chunks):
+        assert binding.segment_plan(inp.B, inp.H, inp.T, inp.dk, inp.dv) == chunks
+        _check(inp, ref, "tcgen05")
+
+
+@pytest.mark.parametrize("level,chunks", [(8, 2), (9, 2), (10, 4), (12, 4), (13, 8), (14, 4)])
+def test_segments_one_hot_levels(level, chunks):
+    # one level at a time with no decay, T = 16384: levels 8 + b >= 8 + log2(chunks) come
+    # entirely from pre-filled blocks, the lower ones from the walk's own merges
+    w = I.shrink(W["t8k_d64_bf16"], B=1, H=1, T=16384)
+    inp = I.make_inputs(w, seed=32, log_a_mode="zero", lam_mode="onehot", lam_level=level)
+    ref = O.llattn_recurrent(inp)
+    with _forced_segments(chunks):
+        _check(inp, ref, "tcgen05")
+
+
+def test_segments_packed_batch():
+    w = I.Workload("vl_seg", B=6, H=2, T=5000, dk=64, dv=64, dtype="bf16", varlen=True)
+    inp = I.make_inputs(w, seed=33, log_a_mode="slow",
+                        lengths=np.array([5000, 1, 0, 129, 4096, 2600]))
+    ref = O.llattn_recurrent(inp)
+    for chunks in (2, 8):
+        with _forced_segments(chunks):
+            _check(inp, ref, "tcgen05")
+    _check(inp, ref, "tcgen05")   # the automatic plan
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64)])
+def test_head_dims_128_on_tensor_cores(dk, dv):
+    # d_k = 128: two 64-column passes, the second adding into out; d_v = 128: two value tiles
+    w = I.Workload("d128", B=1, H=2, T=3000, dk=dk, dv=dv, dtype="bf16")
+    for mode in ("slow", "dist"):
+        inp = I.make_inputs(w, seed=34, log_a_mode=mode)
+        ref = O.llattn_recurrent(inp)
+        _check(inp, ref, "tcgen05")
+        with _forced_segments(4):
+            _check(inp, ref, "tcgen05")
+
+
+def test_long_context_d128_deep_levels():
+    # the 64K-token, d = 128 workload's own decay at T = 32768 (256 chunks, nine chunk levels),
+    # one head, every output against the oracle, automatic segments
+    w = I.shrink(W["t64k_d128_bf16"], H=1, T=32768)
+    inp = I.make_inputs(w, seed=35)
+    ref = O.llattn_recurrent(inp)
+    assert binding.segment_plan(inp.B, inp.H, inp.T, inp.dk, inp.dv) > 0
+    _check(inp, ref, "tcgen05")
