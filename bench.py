@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--segment-chunks", type=int, default=0,
+                    help="force the tensor-core path's segment length in chunks (0: automatic)")
     ap.add_argument("--pass", dest="which", choices=["fwd", "bwd"], default="fwd",
                     help="bwd times the backward pass (gradients of all inputs) instead")
     return ap.parse_args()
@@ -474,6 +476,10 @@ def run_ours(args, w, rank, world, local_rank):
         binding.forward(q, k, v, la, lm, cu_seqlens=cu, T=inp.T, out=out, path=path, chunk=chunk,
                         workspace=ws)
 
+    seg_chunks = 0
+    if path == "tcgen05":
+        seg_chunks = binding.segment_plan(inp.B, inp.H, inp.T, inp.dk, inp.dv, cu is not None)
+
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -535,8 +541,9 @@ def run_ours(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": workload_config(w, chunk, path), "roofline": roof,
-        "gpu_launches": launches, "clocks": clk,
+        "config": {**workload_config(w, chunk, path),
+                   **({"segment_chunks": seg_chunks} if path == "tcgen05" else {})},
+        "roofline": roof, "gpu_launches": launches, "clocks": clk,
     }
 
     # end to end through the host-buffer entry point (pinned host memory)
@@ -1025,16 +1032,216 @@ def run_bwd(args, w, rank, world, local_rank):
     return line
 
 
+# ---------------------------------------------------------------------------------------------
+# Log-Linear Gated DeltaNet forward
+# ---------------------------------------------------------------------------------------------
+GDN_METRIC = "log-linear gated deltanet fwd tokens/s (1×B200)"
+
+
+def gdn_algorithmic(w, lengths):
+    """Bytes: read q, k, v (input type), log_alpha, beta, lam (fp32); write out (fp32).  FLOPs of
+    the recurrent form: at token t every occupied level l >= 1 (popcount(t) of them) takes the
+    transition (k . s and the rank-1 update: 4 d_k d_v), the write is 2 d_k d_v, and each of the
+    popcount(t) + 1 levels read out costs 2 d_k d_v."""
+    esz = 2 if w.dtype == "bf16" else 4
+    per = (2 * w.dk + w.dv) * esz + 4 + 4 + 4 * w.L + 4 * w.dv
+    flops = 0
+    for n in lengths:
+        pc = sum(bin(t).count("1") for t in range(n))
+        flops += (4 * pc + 2 * n + 2 * (pc + n)) * w.dk * w.dv
+    return per * sum(lengths) * w.H, flops * w.H, per
+
+
+def run_gdn(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from hierarchical_fenwick_state_b200 import binding
+    from hierarchical_fenwick_state_b200 import inputs as I
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    inp = I.make_gdn_inputs(w, seed=rank_seed(args.seed, rank))
+    dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    t = {n: torch.from_numpy(getattr(inp, n)).to(dev) for n in ("q", "k", "v", "log_a", "beta", "lam")}
+    for n in ("q", "k", "v"):
+        t[n] = t[n].to(dt)
+    out = torch.empty(inp.v.shape, dtype=torch.float32, device=dev)
+    lengths = [n for _, n in inp.seq_slices()]
+    total_tokens = int(sum(lengths))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        binding.gdn_forward(t["q"], t["k"], t["v"], t["log_a"], t["beta"], t["lam"], out=out)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    binding.profile_read(reset=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    binding.profile(True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    binding.profile(False)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    main_ms, main_n, launches = binding.profile_read(reset=True)
+    if binding.device_status(clear=True):
+        raise RuntimeError("device status flags set after the timed region")
+    ms_step = ms_total / args.steps
+    value = total_tokens * world / (ms_step / 1000.0)
+    hbm_gbs, _, peak_kind = measured_peaks()
+    abytes, aflops, per_tok = gdn_algorithmic(w, lengths)
+    main_avg_s = (main_ms / main_n) / 1000.0 if main_n else ms_step / 1000.0
+    alu = alu_peak_tflops()
+    if abytes / (hbm_gbs * 1e9) >= aflops / (alu * 1e12):
+        roof = {"bound": "hbm", "achieved": abytes / main_avg_s / 1e9, "peak": hbm_gbs,
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "alu", "achieved": aflops / main_avg_s / 1e12, "peak": alu,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["peak_source"] = ("derived fp32 FMA peak: 148 SMs x 128 lanes x 2 x 1965 MHz"
+                           if roof["bound"] == "alu" else
+                           (f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                            else "profiling-recipe fallback"))
+    roof["kernel"] = f"gdn:{w.name}"
+    roof["algorithmic_bytes_per_launch"] = abytes
+    roof["algorithmic_flops_per_launch"] = aflops
+    roof["main_kernel_ms"] = main_avg_s * 1000.0
+    cfg = workload_config(w, None, "cuda cores (recurrent form)")
+    cfg["beta"] = "sigmoid(N(0,1))"
+    cfg["log_a"] = f"log alpha = -exp(N({w.log_a_mu},0.5))"
+    line = {
+        "metric": GDN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic", "config": cfg,
+        "roofline": roof, "gpu_launches": launches, "clocks": clk,
+    }
+    if not args.no_e2e:
+        # per step: inputs up from pinned host memory, the forward, out back
+        if inp.dtype == "bf16":
+            hs = {n: torch.from_numpy(I.bf16_bits(getattr(inp, n)).view(np.int16)).pin_memory()
+                  for n in ("q", "k", "v")}
+        else:
+            hs = {n: torch.from_numpy(getattr(inp, n)).pin_memory() for n in ("q", "k", "v")}
+        for n in ("log_a", "beta", "lam"):
+            hs[n] = torch.from_numpy(getattr(inp, n)).pin_memory()
+        hout = torch.empty(inp.v.shape, dtype=torch.float32).pin_memory()
+        ds = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in hs.items()}
+        h2d = sum(x.numel() * x.element_size() for x in hs.values())
+
+        def e2e_step():
+            for n in hs:
+                ds[n].copy_(hs[n], non_blocking=True)
+            qd, kd, vd = ((ds[n].view(torch.bfloat16) if inp.dtype == "bf16" else ds[n])
+                          for n in ("q", "k", "v"))
+            binding.gdn_forward(qd, kd, vd, ds["log_a"], ds["beta"], ds["lam"], out=out)
+            hout.copy_(out, non_blocking=True)
+            stream.synchronize()
+
+        e2e_step()
+        n_e2e = max(3, min(args.steps, 10))
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1000.0 / n_e2e, dist, dev)
+        line["e2e"] = {"value": total_tokens * world / e2e_s, "unit": "tokens/s",
+                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4),
+                       "steps": n_e2e, "entry": "llattn_gdn_fwd, inputs from pinned host memory"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        start, n = inp.seq_slices()[0]
+        heads = min(inp.H, 4)
+        sl = slice(start, start + n)
+        q_ = inp.q.reshape(-1, inp.H, inp.dk)[sl, :heads].transpose(1, 0, 2)
+        k_ = inp.k.reshape(-1, inp.H, inp.dk)[sl, :heads].transpose(1, 0, 2)
+        v_ = inp.v.reshape(-1, inp.H, inp.dv)[sl, :heads].transpose(1, 0, 2)
+        la_ = inp.log_a.reshape(-1, inp.H)[sl, :heads].T
+        b_ = inp.beta.reshape(-1, inp.H)[sl, :heads].T
+        lm_ = inp.lam.reshape(-1, inp.H, inp.L)[sl, :heads].transpose(1, 0, 2)
+        t0 = time.perf_counter()
+        O.gdn_recurrent_seq(q_, k_, v_, la_, b_, lm_)
+        dts = time.perf_counter() - t0
+        line["cpu_baseline"] = {
+            "value": n * (heads / inp.H) / dts, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"recurrent fp64 Gated DeltaNet oracle, 1 sequence x {heads} of {inp.H} "
+                      f"heads x {n} tokens batched, {dts:.2f} s, numpy", "host": _host_info()}
+    return line
+
+
+def run_gdn_reference(args, w, rank, world):
+    """The Gated DeltaNet oracle (recurrent form) on the host: one sequence x 4 heads per step."""
+    import numpy as np
+    import oracle as O
+    from hierarchical_fenwick_state_b200 import inputs as I
+    if rank != 0:
+        return None
+    inp = I.make_gdn_inputs(w, seed=args.seed)
+    start, n = inp.seq_slices()[0]
+    heads = min(inp.H, 4)
+    sl = slice(start, start + n)
+    arrs = (inp.q.reshape(-1, inp.H, inp.dk)[sl, :heads].transpose(1, 0, 2),
+            inp.k.reshape(-1, inp.H, inp.dk)[sl, :heads].transpose(1, 0, 2),
+            inp.v.reshape(-1, inp.H, inp.dv)[sl, :heads].transpose(1, 0, 2),
+            inp.log_a.reshape(-1, inp.H)[sl, :heads].T, inp.beta.reshape(-1, inp.H)[sl, :heads].T,
+            inp.lam.reshape(-1, inp.H, inp.L)[sl, :heads].transpose(1, 0, 2))
+    arrs = tuple(np.ascontiguousarray(a) for a in arrs)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        O.gdn_recurrent_seq(*arrs)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    dt = statistics.mean(times)
+    value = n * (heads / inp.H) / dt
+    desc = (f"recurrent fp64 Gated DeltaNet oracle, 1 sequence x {heads} of {inp.H} heads x {n} "
+            f"tokens batched, {dt:.2f} s per step, numpy")
+    return {
+        "metric": GDN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * dt,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference", "config": workload_config(w, None, None),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc, "host": _host_info()},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     args = parse()
     from hierarchical_fenwick_state_b200 import inputs as I
     decoding = args.workload in I.DECODE_WORKLOADS
-    w = I.DECODE_WORKLOADS[args.workload] if decoding else I.WORKLOADS[args.workload]
+    gdn = args.workload in I.GDN_WORKLOADS
+    w = (I.DECODE_WORKLOADS if decoding else I.GDN_WORKLOADS if gdn else I.WORKLOADS)[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        if args.which == "bwd" and not decoding:
+        if gdn:
+            line = run_gdn_reference(args, w, rank, world)
+        elif args.which == "bwd" and not decoding:
             line = run_bwd_reference(args, w, rank, world)
         else:
             line = (run_decode_reference if decoding else run_reference)(args, w, rank, world)
@@ -1049,8 +1256,13 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.segment_chunks:
+        from hierarchical_fenwick_state_b200 import binding
+        binding.set_segment_chunks(args.segment_chunks)
     try:
-        if args.which == "bwd" and not decoding:
+        if gdn:
+            line = run_gdn(args, w, rank, world, local_rank)
+        elif args.which == "bwd" and not decoding:
             line = run_bwd(args, w, rank, world, local_rank)
         else:
             line = (run_decode if decoding else run_ours)(args, w, rank, world, local_rank)

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 
 #include "../../include/llattn.h"
@@ -1657,15 +1658,23 @@ SegPlan seg_plan(int nseq, int H, int T, int dk, int dv, bool varlen) {
   }
   const int vh = H * (dv / kD);
   const int nsm = sm_count();
-  const double per = varlen ? 0.5 : 1.0;
   auto waves = [&](long long items) { return (double)((items + nsm - 1) / nsm); };
-  double best = waves((long long)nseq * vh) * (nch + 2);
+  // dense: equal items, so whole waves; packed: lengths spread over [0, T], so the work of the
+  // items (at half the bound each, with ~3 steps of fixed cost per item) spread over the SMs,
+  // plus the longest item
+  auto estimate = [&](int len, long long per_seq, double pre) {
+    if (!varlen) return waves((long long)nseq * vh * per_seq) * (len + 2) + pre;
+    const double avg = 0.5 * nch;
+    const double items = std::ceil(avg / len);
+    return (double)nseq * vh * (avg + 3.0 * items) / nsm + len + pre;
+  };
+  double best = estimate(nch, 1, 0.0);
   for (int g = 1; (1 << g) < nch; ++g) {
     const int nseg = (nch + (1 << g) - 1) >> g;
     if (chunk_levels(nseg) > 8) continue;   // the counter over segments keeps <= 8 levels
-    const long long items = (long long)nseq * vh * ((long long)(per * nch + (1 << g) - 1) >> g);
+    const double per = varlen ? 0.5 : 1.0;
     const double pre = 2.0 + (double)nseq * vh * (per * nch) / (8.0 * nsm);
-    const double est = waves(items) * ((1 << g) + 2) + pre;
+    const double est = estimate(1 << g, nseg, pre);
     if (est < best) {
       best = est;
       pl.g = g;

@@ -76,6 +76,15 @@ WORKLOADS = {
 }
 HEADLINE = "t8k_d64_bf16"
 
+# Log-Linear Gated DeltaNet forward: the same shapes and distributions (log_a is log alpha),
+# plus beta = sigmoid(N(0, 1)) per (token, head) from make_gdn_inputs.
+GDN_WORKLOADS = {
+    "gdn_t2k_d64_bf16": Workload("gdn_t2k_d64_bf16", B=2, H=16, T=2048, dk=64, dv=64,
+                                 dtype="bf16"),
+    "gdn_t8k_d64_bf16": Workload("gdn_t8k_d64_bf16", B=4, H=32, T=8192, dk=64, dv=64,
+                                 dtype="bf16"),
+}
+
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding bf16 values."""
