@@ -1234,7 +1234,8 @@ def main():
     from hierarchical_fenwick_state_b200 import inputs as I
     decoding = args.workload in I.DECODE_WORKLOADS
     gdn = args.workload in I.GDN_WORKLOADS
-    w = (I.DECODE_WORKLOADS if decoding else I.GDN_WORKLOADS if gdn else I.WORKLOADS)[args.workload]
+    w = (I.DECODE_WORKLOADS if decoding else I.GDN_WORKLOADS if gdn else
+         I.PROFILE_WORKLOADS if args.workload in I.PROFILE_WORKLOADS else I.WORKLOADS)[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

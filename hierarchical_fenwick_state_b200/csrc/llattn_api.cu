@@ -633,7 +633,7 @@ llattn_status llattn_decode_step(int in_dtype, const void* q, const void* k, con
 llattn_status llattn_bwd_workspace_bytes(int B, int H, int T, int dk, int dv, size_t* bytes) {
   if (!bytes) return LLATTN_ERR_ARG;
   if (B < 0 || H < 0 || T < 0 || T > (1 << 24) || H > 65535 || B > 65535) return LLATTN_ERR_SHAPE;
-  if (dk != dv || (dk != 32 && dk != 64)) return LLATTN_ERR_SHAPE;
+  if (dk != dv || (dk != 32 && dk != 64 && dk != 128)) return LLATTN_ERR_SHAPE;
   *bytes = (B == 0 || H == 0 || T == 0) ? 0 : llattn::bwd_workspace_bytes(B, H, T);
   return LLATTN_OK;
 }

@@ -33,6 +33,8 @@
 
 #include <cstdint>
 
+#include <atomic>
+
 #include "../../include/llattn.h"
 #include "llattn_bwd.h"
 #include "llattn_common.cuh"
@@ -67,14 +69,25 @@ __global__ void bwd_prefix_g(BwdProblem p, double* g) {
 }
 
 // ---- levels 0..5: dense 32 x 32 tiles ----
+// Dynamic shared memory of the dense tile kernel (over the 48 KB static limit at D = 128).
+template <int D>
+constexpr size_t dense_smem_bytes() {
+  return kTile * sizeof(double) + (4 * kTile * (D + 1) + 3 * kTile * (kTile + 1) +
+                                   kTile * kDenseLevels) * sizeof(float);
+}
+
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kThreads) bwd_dense_tile(BwdProblem p, const double* g) {
-  __shared__ float s_q[kTile][D + 1], s_k[kTile][D + 1], s_v[kTile][D + 1], s_do[kTile][D + 1];
-  __shared__ float s_pm[kTile][kTile + 1];  // (do_i . v_j) M[i, j]
-  __shared__ float s_pa[kTile][kTile + 1];  // (q_i . k_j) M[i, j]
-  __shared__ float s_x[kTile][kTile + 1];   // (do_i . v_j)(q_i . k_j) exp(g_i - g_j)
-  __shared__ double s_g[kTile];
-  __shared__ float s_lam[kTile][kDenseLevels];
+  extern __shared__ __align__(16) unsigned char dsm[];
+  double* s_g = reinterpret_cast<double*>(dsm);                          // [kTile]
+  float (*s_q)[D + 1] = reinterpret_cast<float (*)[D + 1]>(dsm + kTile * sizeof(double));
+  float (*s_k)[D + 1] = s_q + kTile;
+  float (*s_v)[D + 1] = s_k + kTile;
+  float (*s_do)[D + 1] = s_v + kTile;
+  float (*s_pm)[kTile + 1] = reinterpret_cast<float (*)[kTile + 1]>(s_do + kTile);  // (do_i . v_j) M
+  float (*s_pa)[kTile + 1] = s_pm + kTile;   // (q_i . k_j) M[i, j]
+  float (*s_x)[kTile + 1] = s_pa + kTile;    // (do_i . v_j)(q_i . k_j) exp(g_i - g_j)
+  float (*s_lam)[kDenseLevels] = reinterpret_cast<float (*)[kDenseLevels]>(s_x + kTile);
 
   const int tile = blockIdx.x, h = blockIdx.y, sq = blockIdx.z, tid = threadIdx.x;
   const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
@@ -156,14 +169,28 @@ __global__ void __launch_bounds__(kThreads) bwd_dense_tile(BwdProblem p, const d
 }
 
 // ---- one level >= 6: the rank-d interaction of each aligned block's halves ----
+// Dynamic shared memory of the level kernel.  Up to D = 64 the staged rows of phase 1 share
+// space with S and U, and each thread holds both states' accumulators; at D = 128 (64
+// accumulators per state per thread) S is stored after its pass so U can reuse the registers,
+// which needs the staging space apart from S.
+template <int D>
+__host__ __device__ constexpr bool level_split() { return D > 64; }
+template <int D>
+constexpr size_t level_smem_bytes() {
+  return (32 + 2 * D * (D + 1) + (level_split<D>() ? 2 * 32 * D : 0)) * sizeof(float);
+}
+
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kThreads) bwd_level_block(BwdProblem p, const double* g, int lvl) {
   constexpr int R = D * D / kThreads;  // state elements per thread
   constexpr int E = D / 8;             // elements per lane of an 8-lane token group
-  __shared__ float s_mem[2 * D * (D + 1)];  // phase 1: staged rows; phase 2: S and U
-  __shared__ float s_w[32];
-  float (*s_x)[D] = reinterpret_cast<float (*)[D]>(s_mem);               // [32][D]
-  float (*s_y)[D] = reinterpret_cast<float (*)[D]>(s_mem + 32 * D);      // [32][D]
+  constexpr bool kSplit = level_split<D>();
+  extern __shared__ __align__(16) float lsm[];
+  float* s_w = lsm;                                                       // [32]
+  float* s_mem = lsm + 32;              // phase 2: S and U; phase 1: staged rows (unless kSplit)
+  float* s_stage = kSplit ? s_mem + 2 * D * (D + 1) : s_mem;
+  float (*s_x)[D] = reinterpret_cast<float (*)[D]>(s_stage);              // [32][D]
+  float (*s_y)[D] = reinterpret_cast<float (*)[D]>(s_stage + 32 * D);     // [32][D]
   float (*s_S)[D + 1] = reinterpret_cast<float (*)[D + 1]>(s_mem);       // [D][D+1]
   float (*s_U)[D + 1] = reinterpret_cast<float (*)[D + 1]>(s_mem + D * (D + 1));
 
@@ -189,9 +216,11 @@ __global__ void __launch_bounds__(kThreads) bwd_level_block(BwdProblem p, const 
   const double gm = g[grow(mid - 1)];
 
   // phase 1: S over the left half, U over the right half
-  float accS[R], accU[R];
+  float accS[R], accU[kSplit ? 1 : R];
 #pragma unroll
-  for (int r = 0; r < R; ++r) accS[r] = accU[r] = 0.f;
+  for (int r = 0; r < R; ++r) accS[r] = 0.f;
+#pragma unroll
+  for (int r = 0; r < (kSplit ? 1 : R); ++r) accU[r] = 0.f;
   for (int pass = 0; pass < 2; ++pass) {
     const int b0 = pass == 0 ? lo : mid, b1 = pass == 0 ? lend : rend;
     for (int base = b0; base < b1; base += 32) {
@@ -222,18 +251,30 @@ __global__ void __launch_bounds__(kThreads) bwd_level_block(BwdProblem p, const 
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           const int e = tid + r * kThreads, a = e / D, b = e % D;
-          if (pass == 0) accS[r] = fmaf(s_x[i][a], s_y[i][b], accS[r]);
+          if (kSplit || pass == 0) accS[r] = fmaf(s_x[i][a], s_y[i][b], accS[r]);
           else accU[r] = fmaf(s_x[i][a], s_y[i][b], accU[r]);
         }
       }
       __syncthreads();
     }
-  }
+    if (kSplit) {
+      // this pass's state goes to its own region; the registers start over for the next one
+      float (*dst)[D + 1] = pass == 0 ? s_S : s_U;
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int e = tid + r * kThreads, a = e / D, b = e % D;
-    s_S[a][b] = accS[r];
-    s_U[a][b] = accU[r];
+      for (int r = 0; r < R; ++r) {
+        const int e = tid + r * kThreads, a = e / D, b = e % D;
+        dst[a][b] = accS[r];
+        accS[r] = 0.f;
+      }
+    }
+  }
+  if (!kSplit) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = tid + r * kThreads, a = e / D, b = e % D;
+      s_S[a][b] = accS[r];
+      s_U[a][b] = accU[kSplit ? 0 : r];
+    }
   }
   __syncthreads();
 
@@ -357,13 +398,29 @@ __global__ void __launch_bounds__(kThreads) bwd_suffix_scan(BwdProblem p) {
 
 template <typename Tin, int D>
 cudaError_t launch(const BwdProblem& p, double* g, cudaStream_t st) {
+  // the dynamic shared-memory opt-in is a per-device attribute of each kernel
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load()) {
+    if ((e = cudaFuncSetAttribute(bwd_dense_tile<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)dense_smem_bytes<D>())) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_level_block<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)level_smem_bytes<D>())) != cudaSuccess)
+      return e;
+    attr_set[dev].store(true);
+  }
   const dim3 seqs(p.H, p.nseq);
   bwd_prefix_g<<<seqs, 32, 0, st>>>(p, g);
-  bwd_dense_tile<Tin, D><<<dim3((p.T + kTile - 1) / kTile, p.H, p.nseq), kThreads, 0, st>>>(p, g);
+  bwd_dense_tile<Tin, D><<<dim3((p.T + kTile - 1) / kTile, p.H, p.nseq), kThreads,
+                           dense_smem_bytes<D>(), st>>>(p, g);
   int n = 2;
   for (int lvl = kDenseLevels; lvl < p.L; ++lvl, ++n) {
     const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
-    bwd_level_block<Tin, D><<<dim3(nblk, p.H, p.nseq), kThreads, 0, st>>>(p, g, lvl);
+    bwd_level_block<Tin, D><<<dim3(nblk, p.H, p.nseq), kThreads, level_smem_bytes<D>(), st>>>(
+        p, g, lvl);
   }
   bwd_dg<Tin, D><<<dim3((p.T + kThreads / 32 - 1) / (kThreads / 32), p.H, p.nseq), kThreads, 0,
                    st>>>(p);
@@ -379,9 +436,11 @@ cudaError_t bwd(const BwdProblem& p, void* ws, cudaStream_t st) {
   main_kernel_begin(st);
   cudaError_t e;
   if (p.in_dtype == LLATTN_BF16)
-    e = p.d == 32 ? launch<__nv_bfloat16, 32>(p, g, st) : launch<__nv_bfloat16, 64>(p, g, st);
+    e = p.d == 32 ? launch<__nv_bfloat16, 32>(p, g, st)
+                  : p.d == 64 ? launch<__nv_bfloat16, 64>(p, g, st) : launch<__nv_bfloat16, 128>(p, g, st);
   else
-    e = p.d == 32 ? launch<float, 32>(p, g, st) : launch<float, 64>(p, g, st);
+    e = p.d == 32 ? launch<float, 32>(p, g, st)
+                  : p.d == 64 ? launch<float, 64>(p, g, st) : launch<float, 128>(p, g, st);
   main_kernel_end(st);
   return e;
 }

@@ -16,6 +16,12 @@
 // column of every level state, each lane holding d_k / 32 rows of it in registers, and
 // the dot products k . s and q . s are warp reductions.  A CTA of eight warps takes eight
 // columns of one (sequence, head) and walks the sequence token by token.
+//
+// A level with no bucket holds an all-zero state, and the transition keeps it zero, so the
+// transition runs over all levels without branches.  Their 16 dot products k . s_l are then
+// reduced together: a butterfly that halves the set of values each lane carries at every
+// step (16 shuffles in all, 5 dependent steps), after which lanes 2i and 2i + 1 hold the
+// total of level i + 1, and one shuffle per level brings it back to every lane.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -36,6 +42,81 @@ __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
+}
+
+// Sums of 16 values over the warp: v[i] per lane in, the total of value i on every lane out.
+// Step with offset o (16, 8, 4, 2) keeps half of the values each lane carries - the upper half
+// where lane bit log2(o) is set - adding the partner's copy of that half and sending it the
+// other half; the last step (offset 1) completes the sum.  Lanes 2i, 2i + 1 then hold total i.
+__device__ __forceinline__ void warp_sum16(float (&v)[16], int lane) {
+  const unsigned full = 0xffffffffu;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = lane & 16;
+    const float keep = up ? v[i + 8] : v[i], send = up ? v[i] : v[i + 8];
+    v[i] = keep + __shfl_xor_sync(full, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = lane & 8;
+    const float keep = up ? v[i + 4] : v[i], send = up ? v[i] : v[i + 4];
+    v[i] = keep + __shfl_xor_sync(full, send, 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = lane & 4;
+    const float keep = up ? v[i + 2] : v[i], send = up ? v[i] : v[i + 2];
+    v[i] = keep + __shfl_xor_sync(full, send, 4);
+  }
+  {
+    const bool up = lane & 2;
+    const float keep = up ? v[1] : v[0], send = up ? v[0] : v[1];
+    v[0] = keep + __shfl_xor_sync(full, send, 2);
+  }
+  v[0] += __shfl_xor_sync(full, v[0], 1);
+  const float tot = v[0];   // total of value (lane >> 1) & 15
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __shfl_sync(full, tot, 2 * i);
+}
+
+// Promotion: levels 0..m merge into level m + 1 and empty (m = trailing one bits of t).  A
+// switch on m (uniform over the warp) keeps every register index a constant.
+template <int R, int M>
+__device__ __forceinline__ void promote(float (&s)[kGdnMaxLev][R]) {
+  float sum[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) sum[r] = 0.f;
+#pragma unroll
+  for (int l = 0; l <= M; ++l)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      sum[r] += s[l][r];
+      s[l][r] = 0.f;
+    }
+#pragma unroll
+  for (int r = 0; r < R; ++r) s[M + 1][r] = sum[r];
+}
+
+template <int R>
+__device__ __forceinline__ void promote_m(float (&s)[kGdnMaxLev][R], int m) {
+  switch (m) {
+    case 0: promote<R, 0>(s); break;
+    case 1: promote<R, 1>(s); break;
+    case 2: promote<R, 2>(s); break;
+    case 3: promote<R, 3>(s); break;
+    case 4: promote<R, 4>(s); break;
+    case 5: promote<R, 5>(s); break;
+    case 6: promote<R, 6>(s); break;
+    case 7: promote<R, 7>(s); break;
+    case 8: promote<R, 8>(s); break;
+    case 9: promote<R, 9>(s); break;
+    case 10: promote<R, 10>(s); break;
+    case 11: promote<R, 11>(s); break;
+    case 12: promote<R, 12>(s); break;
+    case 13: promote<R, 13>(s); break;
+    case 14: promote<R, 14>(s); break;
+    default: promote<R, 15>(s); break;   // m <= 15 for t < 65536
+  }
 }
 
 template <typename TIn, int R>   // R = d_k / 32 rows of each column per lane
@@ -59,68 +140,76 @@ gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     for (int r = 0; r < R; ++r) s[l][r] = 0.f;
   uint32_t live = 0;   // bit l: level l holds a state (the binary counter of positions)
 
-  for (int t = 0; t < sp.len; ++t) {
-    const long long tok = sp.start + t;
-    const long long base = tok * H + h;
-    float kr[R], qr[R];
+  // the inputs of token t are loaded during token t - 1 (their latency hides behind its work);
+  // lane l holds lam[t, l] (one coalesced load), shuffled to every lane by level
+  float kr[R], qr[R], a_t = 0.f, b_t = 0.f, v_t = 0.f, lam_t = 0.f;
+  auto load = [&](int t, float (&kk)[R], float (&qq)[R], float& aa, float& bb, float& vv, float& ll) {
+    const long long base = (sp.start + t) * H + h;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      kr[r] = ld_in(k + base * DK + r * 32 + lane);
-      qr[r] = ld_in(q + base * DK + r * 32 + lane);
+      kk[r] = ld_in(k + base * DK + r * 32 + lane);
+      qq[r] = ld_in(q + base * DK + r * 32 + lane);
     }
-    const float a = __expf(__ldg(log_alpha + base));
-    const float b = __ldg(beta + base);
-    const float vj = ld_in(v + base * dv + col);
-    const float* lr = lam + base * L;
-    // 1. transition of the occupied levels (l >= 1; level 0 is rewritten below)
+    aa = __ldg(log_alpha + base);
+    bb = __ldg(beta + base);
+    vv = ld_in(v + base * dv + col);
+    ll = lane < L ? __ldg(lam + base * L + lane) : 0.f;
+  };
+  load(0, kr, qr, a_t, b_t, v_t, lam_t);
+
+  for (int t = 0; t < sp.len; ++t) {
+    float nk[R], nq[R], na = 0.f, nb = 0.f, nv = 0.f, nl = 0.f;
+    if (t + 1 < sp.len) load(t + 1, nk, nq, na, nb, nv, nl);
+    const float a = __expf(a_t), b = b_t;
+    // 1. transition of levels 1..16 (level 0 is rewritten below); empty levels stay zero
+    static_assert(kGdnMaxLev == 17, "the batched reduction takes 16 levels");
+    {
+      float p[16];
 #pragma unroll
-    for (int l = 1; l < kGdnMaxLev; ++l) {
-      if (!((live >> l) & 1u)) continue;
-      float p = 0.f;
+      for (int l = 1; l < kGdnMaxLev; ++l) {
+        p[l - 1] = 0.f;
 #pragma unroll
-      for (int r = 0; r < R; ++r) p += kr[r] * s[l][r];
-      p = warp_sum(p) * b;
+        for (int r = 0; r < R; ++r) p[l - 1] += kr[r] * s[l][r];
+      }
+      warp_sum16(p, lane);
 #pragma unroll
-      for (int r = 0; r < R; ++r) s[l][r] = a * (s[l][r] - p * kr[r]);
+      for (int l = 1; l < kGdnMaxLev; ++l) {
+        const float pb = p[l - 1] * b;
+#pragma unroll
+        for (int r = 0; r < R; ++r) s[l][r] = a * (s[l][r] - pb * kr[r]);
+      }
     }
     // 2. the new token's write
 #pragma unroll
-    for (int r = 0; r < R; ++r) s[0][r] = b * kr[r] * vj;
+    for (int r = 0; r < R; ++r) s[0][r] = b * kr[r] * v_t;
     live |= 1u;
     // 3. readout: sum over occupied levels of lam[t, l] (q . s_l)
     float acc = 0.f;
 #pragma unroll
     for (int l = 0; l < kGdnMaxLev; ++l) {
-      if (!((live >> l) & 1u)) continue;
+      if (!((live >> l) & 1u)) continue;   // uniform over the warp; lam past L is never read
+      const float wl = __shfl_sync(0xffffffffu, lam_t, l);
       float p = 0.f;
 #pragma unroll
       for (int r = 0; r < R; ++r) p += qr[r] * s[l][r];
-      acc += __ldg(lr + l) * p;
+      acc += wl * p;
     }
     acc = warp_sum(acc);
-    if (lane == 0) out[base * dv + col] = acc;
+    if (lane == 0) out[((sp.start + t) * H + h) * dv + col] = acc;
     // 4. promotion: levels 0..m into m + 1, m = trailing one bits of t
     if (t + 1 < sp.len) {
       const int m = __ffs(~t) - 1;
-      float sum[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) sum[r] = 0.f;
-#pragma unroll
-      for (int l = 0; l < kGdnMaxLev; ++l) {
-        if (l <= m) {
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            sum[r] += s[l][r];
-            s[l][r] = 0.f;
-          }
-        }
-      }
-#pragma unroll
-      for (int l = 1; l < kGdnMaxLev; ++l)
-        if (l == m + 1)
-#pragma unroll
-          for (int r = 0; r < R; ++r) s[l][r] = sum[r];
+      promote_m<R>(s, m);
       live = (live & ~((2u << m) - 1u)) | (1u << (m + 1));
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        kr[r] = nk[r];
+        qr[r] = nq[r];
+      }
+      a_t = na;
+      b_t = nb;
+      v_t = nv;
+      lam_t = nl;
     }
   }
 }

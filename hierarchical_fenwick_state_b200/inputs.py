@@ -76,6 +76,13 @@ WORKLOADS = {
 }
 HEADLINE = "t8k_d64_bf16"
 
+# Smaller cases of the benchmark workloads for single-kernel profiler captures (inputs still
+# larger than L2, a few hundred MB on the device); not part of the benchmark matrix.
+PROFILE_WORKLOADS = {
+    "t16k_d128_bf16_h8": Workload("t16k_d128_bf16_h8", B=1, H=8, T=16384, dk=128, dv=128,
+                                  dtype="bf16", log_a_mu=-3.0),
+}
+
 # Log-Linear Gated DeltaNet forward: the same shapes and distributions (log_a is log alpha),
 # plus beta = sigmoid(N(0, 1)) per (token, head) from make_gdn_inputs.
 GDN_WORKLOADS = {

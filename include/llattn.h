@@ -338,7 +338,8 @@ LLATTN_API llattn_status llattn_decode_step(int in_dtype, const void* q, const v
  * zero up to rounding (no gate product contains it).
  *
  * llattn_bwd_workspace_bytes - scratch llattn_bwd needs: B*T*H*8 bytes (fp64 prefix sums of
- * log_a), rounded up to 256.  dk == dv in {32, 64}; other head sizes return LLATTN_ERR_SHAPE.
+ * log_a), rounded up to 256.  dk == dv in {32, 64, 128}; other head sizes return
+ * LLATTN_ERR_SHAPE.
  *
  * llattn_bwd
  *   in_dtype   LLATTN_BF16 or LLATTN_F32: the type of q, k, v and dout (bf16 as uint16 bit

@@ -183,14 +183,15 @@ def test_bwd_workspace_bytes():
     assert binding.bwd_workspace_bytes(4, 32, 8192, 64, 64) == 4 * 32 * 8192 * 8
     assert binding.bwd_workspace_bytes(1, 3, 5, 32, 32) == 256          # rounded up to 256
     assert binding.bwd_workspace_bytes(0, 3, 5, 32, 32) == 0
-    for bad in ((1, 1, 16, 64, 32), (1, 1, 16, 128, 128), (1, 1, -1, 64, 64)):
+    assert binding.bwd_workspace_bytes(1, 2, 700, 128, 128) == (2 * 700 * 8 + 255) // 256 * 256
+    for bad in ((1, 1, 16, 64, 32), (1, 1, 16, 48, 48), (1, 1, -1, 64, 64)):
         with pytest.raises(binding.LLAttnError) as e:
             binding.bwd_workspace_bytes(*bad)
         assert e.value.status == 2
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(dk_dim=32), 2), (dict(dk_dim=128, dv_dim=128), 2), (dict(T=-1), 2),
+    (dict(dk_dim=32), 2), (dict(dk_dim=128, dv_dim=64), 2), (dict(dk_dim=48, dv_dim=48), 2), (dict(T=-1), 2),
     (dict(in_dtype=3), 4),
     (dict(dout=0), 1), (dict(dlam=0), 1),
     (dict(dq=0x10008), 3), (dict(dout=0x6008), 3), (dict(dlog_a=0x40002), 3),

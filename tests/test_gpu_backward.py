@@ -62,6 +62,9 @@ CASES = {
     "t2k_d64_bf16": (I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=2048), "slow"),
     "t1_d64_bf16": (I.shrink(W["t2k_d64_bf16"], B=2, H=1, T=1), "dist"),
     "t33_d32_f32": (I.shrink(W["t256_d32_f32"], B=2, H=1, T=33), "slow"),
+    # d = 128: the dense tile in dynamic shared memory, S and U accumulated one at a time
+    "t700_d128_bf16": (I.shrink(W["t64k_d128_bf16"], B=1, H=2, T=700), "slow"),
+    "t300_d128_f32": (I.Workload("b128f", B=2, H=1, T=300, dk=128, dv=128, dtype="f32"), "dist"),
 }
 
 
