@@ -25,6 +25,7 @@ EXPORTS = (
     "llattn_fwd_noalloc", "llattn_decode_state_bytes", "llattn_decode_step",
     "llattn_bwd_workspace_bytes", "llattn_bwd", "llattn_fwd_bf16", "llattn_stream_status",
     "llattn_segment_plan", "llattn_set_segment_chunks", "llattn_gdn_fwd",
+    "llattn_prefill_state",
 )
 
 NOALLOC_SCRATCH_BYTES = 32 << 20  # LLATTN_NOALLOC_SCRATCH_BYTES
@@ -76,6 +77,8 @@ def lib():
     L.llattn_decode_state_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
     L.llattn_decode_step.restype = i
     L.llattn_decode_step.argtypes = [i, vp, vp, vp, f_p, f_p, i_p, f_p, f_p, i, i, i, i, i, vp]
+    L.llattn_prefill_state.restype = i
+    L.llattn_prefill_state.argtypes = [i, vp, vp, f_p, f_p, i, i, i, i, i, i, i_p, vp]
     L.llattn_bwd_workspace_bytes.restype = i
     L.llattn_bwd_workspace_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
     L.llattn_bwd.restype = i
@@ -261,6 +264,26 @@ def decode_step(q, k, v, log_a, lam, pos, state, out, B, H, L, dk, dv, stream=No
                                   int(dk), int(dv), _stream_handle(stream))
     _check(st, "llattn_decode_step")
     return out
+
+
+def prefill_state(k, v, log_a, state, B, H, T, L, dk, dv, cu_seqlens=None, stream=None):
+    """Direct call of llattn_prefill_state: the decoding state of every sequence at the
+    position equal to its length (a prompt's hand-off to decode_step).
+
+    k, v dense [B,T,H,d] or packed [total,H,d] (bf16 or fp32) as the forward takes them,
+    log_a fp32 [..,H], state fp32 of decode_state_bytes(B,H,L,dk,dv) bytes (written),
+    cu_seqlens int32 [B+1] or None."""
+    in_dtype = BF16 if str(k.dtype) == "torch.bfloat16" else F32
+    st = lib().llattn_prefill_state(in_dtype, ctypes.c_void_p(k.data_ptr()),
+                                    ctypes.c_void_p(v.data_ptr()),
+                                    ctypes.c_void_p(log_a.data_ptr()),
+                                    ctypes.c_void_p(state.data_ptr()), int(B), int(H), int(T),
+                                    int(L), int(dk), int(dv),
+                                    ctypes.c_void_p(cu_seqlens.data_ptr())
+                                    if cu_seqlens is not None else None,
+                                    _stream_handle(stream))
+    _check(st, "llattn_prefill_state")
+    return state
 
 
 def bwd_workspace_bytes(B: int, H: int, T: int, dk: int, dv: int) -> int:

@@ -630,6 +630,41 @@ llattn_status llattn_decode_step(int in_dtype, const void* q, const void* k, con
   return LLATTN_OK;
 }
 
+llattn_status llattn_prefill_state(int in_dtype, const void* k, const void* v,
+                                   const float* log_a, float* state, int B, int H, int T, int L,
+                                   int dk, int dv, const int* cu_seqlens, void* stream) {
+  if (in_dtype != LLATTN_F32 && in_dtype != LLATTN_BF16) return LLATTN_ERR_DTYPE;
+  size_t state_bytes = 0;
+  llattn_status s = llattn_decode_state_bytes(B, H, L, dk, dv, &state_bytes);
+  if (s != LLATTN_OK) return s;
+  if (T < 0 || T > (1 << 24)) return LLATTN_ERR_SHAPE;
+  if (B == 0 || H == 0) return LLATTN_OK;  // nothing to compute
+  if (!state) return LLATTN_ERR_ARG;
+  if (T > 0 && (!k || !v || !log_a)) return LLATTN_ERR_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(state, 16) || !aligned(log_a, 4) ||
+      (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return LLATTN_ERR_ALIGN;
+  if (cu_seqlens == nullptr) {   // dense: the inputs' extents are known here
+    const size_t rows = (size_t)B * T * H, esz = in_dtype == LLATTN_BF16 ? 2 : 4;
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(state), s1 = s0 + state_bytes;
+    const struct { const void* p; size_t n; } rng[3] = {
+        {k, rows * dk * esz}, {v, rows * dv * esz}, {log_a, rows * sizeof(float)}};
+    for (const auto& r : rng) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(r.p), a1 = a0 + r.n;
+      if (r.n && a0 < s1 && s0 < a1) return LLATTN_ERR_ARG;
+    }
+  }
+  DeviceState* ds = nullptr;
+  int dev = 0;
+  if ((s = device_state(&ds, &dev)) != LLATTN_OK) return s;
+  const size_t nlev = (size_t)B * H * (size_t)(L - 1) * dk * dv;
+  llattn::PrefillProblem p{in_dtype, k, v, log_a, state, state + nlev, B, H, T, L, dk, dv,
+                           cu_seqlens, ds->status};
+  const cudaError_t e = llattn::prefill_state(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return LLATTN_OK;
+}
+
 llattn_status llattn_bwd_workspace_bytes(int B, int H, int T, int dk, int dv, size_t* bytes) {
   if (!bytes) return LLATTN_ERR_ARG;
   if (B < 0 || H < 0 || T < 0 || T > (1 << 24) || H > 65535 || B > 65535) return LLATTN_ERR_SHAPE;

@@ -30,6 +30,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cooperative_groups.h>
+
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/llattn.h"
@@ -38,6 +41,7 @@
 #include "llattn_internal.h"
 
 namespace llattn {
+namespace cg = cooperative_groups;
 namespace {
 
 constexpr int kThreads = 256;
@@ -193,6 +197,247 @@ cudaError_t launch(const DecodeProblem& p, cudaStream_t st) {
 }
 
 }  // namespace
+
+// ---- the state after a prompt: level l's bucket of tokens, with its pending gate ----
+//
+// For a sequence of n tokens, the next token is at position n, and level l >= 1 holds the tokens
+// s < n with l(n, s) = l: the bucket [lo, hi) = [P 2^l, P 2^l + 2^(l-1)), P = n >> l, present
+// when bit l-1 of n is set ("Partizionamento Gerarchico").  Its state just before n is the sum
+// over the bucket of (prod_{r=s+1..n-1} a_r) k_s v_s^T.  The slot stores that sum gated only to
+// the bucket's last token hi-1, and the gate row holds the rest, sum_{r=hi..n-1} log a_r: the
+// decoding step's lazy gate folds it in at read time, so the stored values stay of the size of
+// one token's k v^T instead of underflowing under a long stretch of decay.
+//
+// Work split.  A cluster of eight CTAs takes one (level, head, sequence); CTA r takes the r-th
+// stretch of the bucket counted from its end, walks it from the end in tiles of 32 tokens and
+// sums f_s k_s v_s^T into a register tile (each thread a dk/16 x dv/16 block: per token it reads
+// dk/16 + dv/16 staged values for dk*dv/256 FMAs).  The factor f_s = exp(D + suffix) <= 1, D the
+// log decay from the tile's end to the bucket's end.  The eight partial states then meet in
+// distributed shared memory: CTA r adds up its eighth of the elements over the ranks in rank
+// order and stores it, so the result does not depend on scheduling.
+namespace {
+
+constexpr int kPfTile = 32;
+constexpr int kPfCluster = 8;
+
+template <int DK, int DV>
+constexpr int prefill_smem_bytes() {
+  return (DK * DV + kPfTile * (DK + DV)) * (int)sizeof(float);
+}
+
+// Sum over the CTA, returned to every thread (s_red: one float per warp; reusable on return).
+__device__ __forceinline__ float block_sum(float x, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = x;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) t += s_red[w];
+  __syncthreads();
+  return t;
+}
+
+// N consecutive floats of shared memory (N in {2, 4, 8}, address aligned to min(N, 4) floats)
+// in 64- or 128-bit loads.
+template <int N>
+__device__ __forceinline__ void ld_smem_vec(float (&x)[N], const float* src) {
+  if constexpr (N == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(src);
+    x[0] = a.x; x[1] = a.y;
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; j += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(src + j);
+      x[j] = a.x; x[j + 1] = a.y; x[j + 2] = a.z; x[j + 3] = a.w;
+    }
+  }
+}
+
+template <typename Tin, int DK, int DV>
+__global__ void __cluster_dims__(kPfCluster, 1, 1) __launch_bounds__(kThreads)
+prefill_kernel(PrefillProblem p) {
+  constexpr int TK = DK / 16, TV = DV / 16;   // the thread's block of the state
+  static_assert(TK * TV * kThreads == DK * DV, "256 threads tile the state");
+  extern __shared__ float4 pf_smem[];
+  float* s_part = reinterpret_cast<float*>(pf_smem);   // [DK][DV] this CTA's partial state
+  float* s_k = s_part + DK * DV;                       // [kPfTile][DK]
+  float* s_v = s_k + kPfTile * DK;                     // [kPfTile][DV]
+  __shared__ float s_f[kPfTile], s_red[kThreads / 32];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int lvl = blockIdx.x / kPfCluster + 1, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int nslot = p.L - 1;
+  const SeqSpan sp = seq_span(b, p.T, p.cu_seqlens, p.status);
+  const int n = sp.len;
+  // both exits below are uniform over the cluster (they depend on the level, head, sequence)
+  if (nslot < 31 && n >= (1 << nslot)) {   // the slots cannot hold position n
+    if (lvl == 1 && rank == 0 && h == 0 && tid == 0) atomicOr(p.status, LLATTN_DEV_DECODE_POS);
+    return;
+  }
+  float* g = p.gate + ((size_t)b * p.H + h) * 2 * nslot;
+  if (!((n >> (lvl - 1)) & 1)) {           // no bucket at this level: nothing pending either
+    if (rank == 0 && tid == 0) g[lvl - 1] = g[nslot + lvl - 1] = 0.f;
+    return;
+  }
+  const int lo = (n >> lvl) << lvl, hi = lo + (1 << (lvl - 1));
+  const int span = ((hi - lo + kPfCluster * kPfTile - 1) / (kPfCluster * kPfTile)) * kPfTile;
+  const int r_hi = max(lo, hi - rank * span), r_lo = max(lo, hi - (rank + 1) * span);
+  const Tin* k = static_cast<const Tin*>(p.k);
+  const Tin* v = static_cast<const Tin*>(p.v);
+  auto row = [&](int t) { return (size_t)(sp.start + t) * p.H + h; };
+
+  if (rank == 0) {   // the pending gate: log decay of the tokens after the bucket, hi .. n-1
+    float part = 0.f;
+    for (int t = hi + tid; t < n; t += kThreads) part += __ldg(p.log_a + row(t));
+    const float d0 = block_sum(part, s_red);
+    if (tid == 0) g[lvl - 1] = g[nslot + lvl - 1] = d0;
+  }
+  // D: log decay from the end of this CTA's stretch to the bucket's last token
+  float D = 0.f;
+  {
+    float part = 0.f;
+    for (int t = r_hi + tid; t < hi; t += kThreads) part += __ldg(p.log_a + row(t));
+    D = block_sum(part, s_red);
+  }
+
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[TK][TV];
+#pragma unroll
+  for (int a = 0; a < TK; ++a)
+#pragma unroll
+    for (int c = 0; c < TV; ++c) acc[a][c] = 0.f;
+
+  // The next tile's rows are loaded into registers while the current one is summed: thread
+  // tid holds float4 number tid + j*256 of the tile's k rows (and of its v rows), warp 0 the
+  // tile's log a (lane i: token t0 + i).  Rows past the stretch read as zeros.
+  constexpr int NK = kPfTile * DK / 4 / kThreads, NV = kPfTile * DV / 4 / kThreads;
+  static_assert(NK >= 1 && NV >= 1, "a tile is at least one float4 per thread");
+  float4 rk[NK], rv[NV];
+  float rla = 0.f;
+  auto fetch = [&](int t0, int m) {
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      const int e = tid + j * kThreads, i = e / (DK / 4), c = 4 * (e % (DK / 4));
+      rk[j] = i < m ? ld4_in(k + row(t0 + i) * DK + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int e = tid + j * kThreads, i = e / (DV / 4), c = 4 * (e % (DV / 4));
+      rv[j] = i < m ? ld4_in(v + row(t0 + i) * DV + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid < 32) rla = tid < m ? __ldg(p.log_a + row(t0 + tid)) : 0.f;
+  };
+  if (r_hi > r_lo) fetch(max(r_lo, r_hi - kPfTile), r_hi - max(r_lo, r_hi - kPfTile));
+
+  for (int t1 = r_hi; t1 > r_lo; t1 -= kPfTile) {
+    const int t0 = max(r_lo, t1 - kPfTile), m = t1 - t0;
+    __syncthreads();   // the previous tile is summed: its staging can be overwritten
+    if (tid < 32) {
+      // factor of token t0 + lane: exp(D + sum of log a over t0+lane+1 .. t1-1), from the
+      // suffix sums x = sum over t0+lane .. t1-1; D then moves past this tile (warp 0 keeps it)
+      float x = rla;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, x, o);
+        if (tid + o < 32) x += y;
+      }
+      s_f[tid] = __expf(D + (x - rla));
+      D += __shfl_sync(0xffffffffu, x, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      const int e = tid + j * kThreads;
+      *reinterpret_cast<float4*>(s_k + (e / (DK / 4)) * DK + 4 * (e % (DK / 4))) = rk[j];
+    }
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int e = tid + j * kThreads;
+      *reinterpret_cast<float4*>(s_v + (e / (DV / 4)) * DV + 4 * (e % (DV / 4))) = rv[j];
+    }
+    __syncthreads();
+    if (t0 > r_lo) fetch(max(r_lo, t0 - kPfTile), t0 - max(r_lo, t0 - kPfTile));
+    for (int i = 0; i < m; ++i) {
+      float kk[TK], vv[TV];
+      ld_smem_vec<TK>(kk, s_k + i * DK + ty * TK);
+      ld_smem_vec<TV>(vv, s_v + i * DV + tx * TV);
+      const float f = s_f[i];
+#pragma unroll
+      for (int a = 0; a < TK; ++a) kk[a] *= f;
+#pragma unroll
+      for (int a = 0; a < TK; ++a)
+#pragma unroll
+        for (int c = 0; c < TV; ++c) acc[a][c] = fmaf(kk[a], vv[c], acc[a][c]);
+    }
+  }
+
+  // partial state to shared memory, then each rank reduces its eighth over the cluster
+#pragma unroll
+  for (int a = 0; a < TK; ++a)
+#pragma unroll
+    for (int c = 0; c < TV; ++c) s_part[(ty * TK + a) * DV + tx * TV + c] = acc[a][c];
+  cluster.sync();
+  constexpr int kShare = DK * DV / 4 / kPfCluster;   // float4s each rank reduces
+  float4* dst = reinterpret_cast<float4*>(p.levels + (((size_t)b * p.H + h) * nslot + (lvl - 1)) *
+                                                         (size_t)DK * DV);
+  for (int e = tid; e < kShare; e += kThreads) {
+    const int idx = rank * kShare + e;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < kPfCluster; ++q) {
+      const float4 x = cluster.map_shared_rank(reinterpret_cast<float4*>(s_part), q)[idx];
+      sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
+    }
+    dst[idx] = sum;
+  }
+  cluster.sync();   // no CTA leaves while another reads its partial
+}
+
+template <typename Tin, int DK, int DV>
+cudaError_t launch_prefill_one(const PrefillProblem& p, cudaStream_t st) {
+  // the dynamic shared-memory opt-in is a per-device attribute of each kernel
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load()) {
+    if ((e = cudaFuncSetAttribute(prefill_kernel<Tin, DK, DV>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  prefill_smem_bytes<DK, DV>())) != cudaSuccess)
+      return e;
+    attr_set[dev].store(true);
+  }
+  const dim3 grid(kPfCluster * (p.L - 1), p.H, p.B);
+  prefill_kernel<Tin, DK, DV><<<grid, kThreads, prefill_smem_bytes<DK, DV>(), st>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename Tin, int DK>
+cudaError_t launch_prefill_dk(const PrefillProblem& p, cudaStream_t st) {
+  switch (p.dv) {
+    case 32: return launch_prefill_one<Tin, DK, 32>(p, st);
+    case 64: return launch_prefill_one<Tin, DK, 64>(p, st);
+    default: return launch_prefill_one<Tin, DK, 128>(p, st);
+  }
+}
+
+template <typename Tin>
+cudaError_t launch_prefill(const PrefillProblem& p, cudaStream_t st) {
+  switch (p.dk) {
+    case 32: return launch_prefill_dk<Tin, 32>(p, st);
+    case 64: return launch_prefill_dk<Tin, 64>(p, st);
+    default: return launch_prefill_dk<Tin, 128>(p, st);
+  }
+}
+
+}  // namespace
+
+cudaError_t prefill_state(const PrefillProblem& p, cudaStream_t st) {
+  if (p.L < 2) return cudaSuccess;   // no level slots
+  count_launch(1);
+  return p.in_dtype == LLATTN_BF16 ? launch_prefill<__nv_bfloat16>(p, st) : launch_prefill<float>(p, st);
+}
 
 cudaError_t decode_step(const DecodeProblem& p, cudaStream_t st) {
   count_launch(1);

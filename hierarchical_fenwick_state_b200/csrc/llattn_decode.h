@@ -30,4 +30,20 @@ inline size_t decode_state_bytes(int B, int H, int L, int dk, int dv) {
 
 cudaError_t decode_step(const DecodeProblem& p, cudaStream_t st);
 
+// The decoding state after a prompt (llattn_prefill_state): every sequence of a dense or packed
+// batch, at the position equal to its length.
+struct PrefillProblem {
+  int in_dtype;          // LLATTN_F32 / LLATTN_BF16: type of k, v
+  const void* k;         // [.., H, dk] token-major, as the forward's inputs
+  const void* v;         // [.., H, dv]
+  const float* log_a;    // [.., H]
+  float* levels;         // the decoding state's level slots [B, H, L-1, dk, dv]
+  float* gate;           // and its gate rows [B, H, 2, L-1]
+  int B, H, T, L, dk, dv;
+  const int* cu_seqlens; // device, or null (dense: every length is T)
+  unsigned int* status;
+};
+
+cudaError_t prefill_state(const PrefillProblem& p, cudaStream_t st);
+
 }  // namespace llattn

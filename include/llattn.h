@@ -99,7 +99,7 @@ enum {
   LLATTN_DEV_SEQ_TOO_LONG = 1u,  /* a varlen sequence was longer than T */
   LLATTN_DEV_WAIT_TIMEOUT = 2u,  /* an mbarrier / pipeline wait hit its iteration limit */
   LLATTN_DEV_BAD_CU_SEQLENS = 4u, /* cu_seqlens decreasing */
-  LLATTN_DEV_DECODE_POS = 8u,    /* llattn_decode_step: a position outside [0, 2^(L-1)) */
+  LLATTN_DEV_DECODE_POS = 8u,    /* decode step or prefill state: a position outside [0, 2^(L-1)) */
   LLATTN_DEV_NONFINITE = 16u     /* tensor-core forward: an output value came out inf or NaN.
                                   * With finite inputs this means an intermediate rounded to
                                   * fp16 (P, V, the decay-scaled K, a level state, Q) left
@@ -320,6 +320,47 @@ LLATTN_API llattn_status llattn_decode_step(int in_dtype, const void* q, const v
                                             const void* v, const float* log_a, const float* lam,
                                             const int* pos, float* state, float* out, int B,
                                             int H, int L, int dk, int dv, void* stream);
+
+/*
+ * llattn_prefill_state - the decoding state after a prompt: for every sequence of a dense or
+ * packed batch, the state llattn_decode_step expects at position n = the sequence's length,
+ * so that decoding continues the prompt (its outputs come from llattn_fwd).
+ *
+ * Log-Linear Attention (gist.science summaries, Italian "Sommario tecnico" section 2,
+ * "Partizionamento Gerarchico"; Spanish "Resumen tecnico" section 2, "Particion Jerarquica"):
+ * seen from position n, the earlier tokens fall into the Fenwick buckets of n: level l >= 1
+ * holds the tokens s < n with l(n, s) = l, i.e. [P 2^l, P 2^l + 2^(l-1)) with P = n >> l,
+ * non-empty exactly when bit l-1 of n is set.  Its state just before n is
+ *   sum over s in that bucket of (prod_{r=s+1..n-1} a_r) k_s v_s^T,   a_r = exp(log_a[r]).
+ * It is written in the decoding state's lazy-gate form: slot l-1 receives the sum gated only
+ * up to the bucket's last token (prod over r = s+1 .. P 2^l + 2^(l-1) - 1), and both gate rows
+ * gate[b, h, 0..1, l-1] receive the log of the rest, sum of log_a[r] over the tokens after the
+ * bucket, so that exp(gate) * slot is the state (the stored values never underflow however
+ * long the decay after the bucket).  Levels without a bucket get gate 0 and keep their slot's
+ * contents (decoding never reads them).
+ *   in_dtype  LLATTN_BF16 (k, v as uint16 bf16 bit patterns) or LLATTN_F32.
+ *   k, v      DEVICE: dense [B, T, H, dk] / [B, T, H, dv], or packed [total, H, dk] /
+ *             [total, H, dv] with cu_seqlens, as llattn_fwd takes them.  log_a [.., H] fp32.
+ *             q and lam are not needed: the state holds no readout.
+ *   state     DEVICE fp32 buffer of llattn_decode_state_bytes(B, H, L, dk, dv), caller-owned,
+ *             laid out as llattn_decode_step describes; the occupied level slots and all
+ *             gate entries of every (sequence, head) are written.  Decoding then starts with
+ *             pos[b] = n.
+ *   cu_seqlens DEVICE int32 [B + 1] or NULL (every length is T).  A length above T is cut
+ *             to T and sets LLATTN_DEV_SEQ_TOO_LONG; a decreasing one sets LLATTN_DEV_BAD_CU_SEQLENS.
+ *   L         the decode state's level count: lengths n must be below 2^(L-1) (a sequence at
+ *             n >= 2^(L-1) is left unwritten and sets LLATTN_DEV_DECODE_POS).
+ *   dk, dv    in {32, 64, 128}.  B, H <= 65535, 0 <= T <= 2^24, 1 <= L <= 32.
+ * Pointers: k, v and state 16-byte aligned, log_a and cu_seqlens 4-byte aligned; state must not
+ * overlap the inputs.  Asynchronous on `stream`; fp32 arithmetic on CUDA cores, one CTA per
+ * (level, head, sequence) walking its bucket from the end (the suffix decay factors are at
+ * most 1).  It reads each prompt token's k and v once per level whose bucket holds it, i.e.
+ * once in all.
+ */
+LLATTN_API llattn_status llattn_prefill_state(int in_dtype, const void* k, const void* v,
+                                              const float* log_a, float* state, int B, int H,
+                                              int T, int L, int dk, int dv,
+                                              const int* cu_seqlens, void* stream);
 
 /*
  * Backward pass: the gradients of sum(dout * out) with respect to q, k, v, log_a and lam, for

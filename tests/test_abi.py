@@ -166,6 +166,35 @@ def test_decode_empty_batches_are_no_ops():
     assert _decode(H=0) == 0
 
 
+def _prefill(**kw):
+    a = dict(in_dtype=1, k=0x2000, v=0x3000, log_a=0x4000, state=0x100000, B=2, H=3, T=40, L=7,
+             dk=64, dv=64, cu=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return binding.lib().llattn_prefill_state(a["in_dtype"], vp(a["k"]), vp(a["v"]),
+                                              vp(a["log_a"]), vp(a["state"]), a["B"], a["H"],
+                                              a["T"], a["L"], a["dk"], a["dv"],
+                                              vp(a["cu"]) if a["cu"] else None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48), 2), (dict(dv=256), 2), (dict(L=0), 2), (dict(L=33), 2), (dict(B=-1), 2),
+    (dict(T=-1), 2), (dict(T=(1 << 24) + 1), 2), (dict(in_dtype=7), 4),
+    (dict(k=0), 1), (dict(log_a=0), 1), (dict(state=0), 1),
+    (dict(k=0x2008), 3), (dict(v=0x3004), 3), (dict(state=0x100004), 3), (dict(log_a=0x4002), 3),
+    (dict(cu=0x5002), 3),
+    # the state overlaps v (2 x 40 x 3 rows of 64 bf16 at 0x3000)
+    (dict(state=0x3100), 1),
+])
+def test_prefill_argument_errors_before_launch(kw, status):
+    assert _prefill(**kw) == status
+
+
+def test_prefill_empty_batches_are_no_ops():
+    assert _prefill(B=0) == 0
+    assert _prefill(H=0) == 0
+
+
 def _bwd(**kw):
     a = dict(in_dtype=1, q=0x1000, k=0x2000, v=0x3000, log_a=0x4000, lam=0x5000, dout=0x6000,
              dq=0x10000, dk=0x20000, dv=0x30000, dlog_a=0x40000, dlam=0x50000, B=1, H=2, T=16,
