@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["llattn_api.cu", "llattn_simt.cu", "llattn_tc.cu", "llattn_noalloc.cu",
-           "llattn_decode.cu", "llattn_bwd.cu", "llattn_gdn.cu"]
+           "llattn_decode.cu", "llattn_bwd.cu", "llattn_bwd_tc.cu", "llattn_gdn.cu"]
 HEADERS = ["llattn_internal.h", "llattn_common.cuh", "llattn_tc_ptx.cuh", "llattn_decode.h",
            "llattn_bwd.h", "llattn_gdn.h"]
 LIB = os.path.join(HERE, "libllattn.so")

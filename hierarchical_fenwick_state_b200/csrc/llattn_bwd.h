@@ -33,4 +33,10 @@ inline size_t bwd_workspace_bytes(int nseq, int H, int T) {
 
 cudaError_t bwd(const BwdProblem& p, void* ws, cudaStream_t st);
 
+// Levels kTcFirstLevel.. on the tensor cores (bf16 inputs, d = 64): one launch per level after
+// the dense tiles and the CUDA-core levels below it; g = the fp64 prefix sums of log_a.
+constexpr int kTcFirstLevel = 7;
+bool bwd_tc_supports(const BwdProblem& p);
+cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st);
+
 }  // namespace llattn

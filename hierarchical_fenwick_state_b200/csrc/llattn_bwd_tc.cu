@@ -1,0 +1,452 @@
+// Backward pass, levels >= 7, on the tensor cores (bf16 inputs, d = 64).
+//
+// Log-Linear Attention (gist.science summaries, Italian "Sommario tecnico" section 2, "Matrici
+// Gerarchiche"): at level l the positions fall into aligned blocks of 2^l tokens, and every key
+// s in a block's left half meets every query t in its right half with weight
+// lam[t, l] exp(g_t - g_s).  With m the last position of the left half the interaction has
+// rank d, and the block needs only
+//
+//   S = sum over left-half s of exp(g_m - g_s) k_s v_s^T             (d x d)
+//   U = sum over right-half t of lam[t, l] exp(g_t - g_m) q_t do_t^T  (d x d)
+//
+// for   w_t = exp(g_t - g_m) S do_t,  dlam[t, l] = q_t . w_t,  dq_t += lam[t, l] w_t,
+//       dk_s += exp(g_m - g_s) U v_s,  dv_s += exp(g_m - g_s) U^T k_s   (dlam = 0 on the left).
+//
+// One CTA takes one block and walks it twice in tiles of 128 tokens.  Pass 1 reduces S and U
+// over the tiles on the tensor cores (K^T V and Q^T dO shapes, M = 64, the token index as the
+// reduction dimension) into TMEM.  Pass 2 multiplies every tile by them: W = dO S^T,
+// DK = V U^T, DV = K U (M = 128 rows per tile), and the epilogue applies the exponential
+// factors, forms dlam and adds into dq, dk, dv.
+//
+// Precision: q, k, v and dO enter as the bf16 values they are.  The operands the method derives
+// (the decay-scaled rows of K and Q, and S, U) are split into a bf16 high part and a bf16
+// remainder, x = hi + lo with |lo| <= 2^-8 |x|, and each product takes both parts (two MMAs into
+// the same fp32 accumulator): about 16 significant bits per operand, so the gradients stay at
+// fp32-accumulation accuracy.  Factors: exp(g_m - g_s) <= 1 on the left half; on the right,
+// exp(g_t - g_m) <= 1 times lam.
+//
+// Loads: whole tiles inside the sequence by TMA (128-byte swizzle, the layout the MMA
+// descriptors read); a tile that runs past the sequence end by plain loads with zero fill, so
+// no load ever leaves the tensors.  Waits are bounded (mbarrier with a time limit; a timeout
+// sets LLATTN_DEV_WAIT_TIMEOUT and the CTA stops issuing work).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "../../include/llattn.h"
+#include "llattn_bwd.h"
+#include "llattn_common.cuh"
+#include "llattn_internal.h"
+#include "llattn_tc_ptx.cuh"
+
+namespace llattn {
+namespace {
+
+using namespace ptx;
+
+constexpr int kC = 128;          // tile rows (tokens)
+constexpr int kD = 64;           // d_k = d_v
+constexpr int kThreads = 256;    // warp w: TMEM lanes 32*(w%4).., column half w/4
+
+// ---- shared memory (bytes from a 1024-byte aligned base) ----
+constexpr uint32_t kTileB = kC * 128;            // 128 rows x 128 B, 128-byte swizzle
+constexpr uint32_t kOffQ = 0, kOffK = kTileB, kOffV = 2 * kTileB, kOffDO = 3 * kTileB;
+constexpr uint32_t kOffQlo = 4 * kTileB, kOffKlo = 5 * kTileB;
+constexpr uint32_t kState = kD * 128;            // 64 rows x 128 B
+constexpr uint32_t kOffShi = 6 * kTileB, kOffSlo = kOffShi + kState;
+constexpr uint32_t kOffUhi = kOffSlo + kState, kOffUlo = kOffUhi + kState;
+constexpr uint32_t kOffDl = kOffUlo + kState;    // dlam partials of column half 1: [128] fp32
+constexpr uint32_t kOffBar = kOffDl + kC * 4;    // [0] loads, [1] MMAs
+constexpr uint32_t kOffMisc = kOffBar + 16;      // [0] TMEM base, [1] abort
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
+
+// ---- TMEM columns ----
+constexpr uint32_t kColS = 0, kColU = 64;        // M = 64 accumulators
+constexpr uint32_t kColW = 128, kColDK = 192, kColDV = 256;   // M = 128 accumulators
+
+constexpr uint32_t kIdescRed = idesc_bf16(64, 64, 1, 1);     // X^T (M contiguous) x Y (N contiguous)
+constexpr uint32_t kIdescKK = idesc_bf16(128, 64, 0, 0);     // rows (K-major) x state rows (K-major)
+constexpr uint32_t kIdescKN = idesc_bf16(128, 64, 0, 1);     // rows (K-major) x state (N contiguous)
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return sdesc_sw128(saddr, 16, 1024); }
+__device__ __forceinline__ uint64_t mndesc(uint32_t saddr) { return sdesc_sw128(saddr, 8192, 1024); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // a -> low 16 bits
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// x = hi + lo: hi = bf16(x) (round to nearest), lo = bf16(x - hi); pairs (a, b), a in the low
+// 16 bits of each word.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf16(a - hf.x, b - hf.y);
+}
+
+__device__ __forceinline__ float2 bf2_at(const uint8_t* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+             const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+             const BwdProblem p, const double* __restrict__ g, int lvl) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int sub = warp & 3, hf = warp >> 2, row = sub * 32 + lane;
+  const uint32_t lane_off = uint32_t(sub * 32) << 16;
+  const int blk = blockIdx.x, h = blockIdx.y, sq = blockIdx.z;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  const int half = 1 << (lvl - 1);
+  const long long a0 = (long long)blk << lvl;
+  if (a0 >= sp.len) return;
+  const int lo = (int)a0, mid = lo + half;
+  const int lend = min(mid, sp.len);                                          // left [lo, lend)
+  const int rend = (int)min((long long)lo + 2 * half, (long long)sp.len);    // right [mid, rend)
+  auto row_of = [&](int t) { return (size_t)(sp.start + t) * p.H + h; };
+  auto grow = [&](int t) { return ((size_t)sq * p.T + t) * p.H + h; };
+  for (int t = lo + tid; t < lend; t += kThreads) p.dlam[row_of(t) * p.L + lvl] = 0.f;
+  if (mid >= sp.len) return;   // no right half: nothing meets at this level
+
+  uint8_t* tq = sm + kOffQ;
+  uint8_t* tk = sm + kOffK;
+  uint8_t* tv = sm + kOffV;
+  uint8_t* tdo = sm + kOffDO;
+  uint8_t* tqlo = sm + kOffQlo;
+  uint8_t* tklo = sm + kOffKlo;
+  uint8_t* shi = sm + kOffShi;
+  uint8_t* slo = sm + kOffSlo;
+  uint8_t* uhi = sm + kOffUhi;
+  uint8_t* ulo = sm + kOffUlo;
+  float* s_dl = reinterpret_cast<float*>(sm + kOffDl);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+
+  if (warp == 0) {
+    tmem_alloc(&misc[0], 512);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+    misc[1] = 0;
+    prefetch_tensormap(&tmq);
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+    prefetch_tensormap(&tmo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const double gm = g[grow(mid - 1)];
+  uint32_t ph_ld = 0u, ph_mma = 0u;
+  int stuck = -1;               // barrier whose wait timed out (its parity in stuck_par)
+  uint32_t stuck_par = 0u;
+  auto bwait = [&](int b, uint32_t& ph) {
+    if (!mbar_wait(&bars[b], ph)) {
+      atomicOr(p.status, LLATTN_DEV_WAIT_TIMEOUT);
+      misc[1] = 1;
+      if (stuck < 0) {
+        stuck = b;
+        stuck_par = ph;
+      }
+    }
+    ph ^= 1u;
+  };
+
+  // One tile of 128 tokens from t0: the tensors a pass needs.  Whole tiles inside the sequence
+  // come by TMA (returns true: wait on bars[0]); a tile running past the sequence end by plain
+  // loads of its rows, the rest zero.
+  auto load = [&](int t0, bool nq, bool nk, bool nv, bool ndo) {
+    if (t0 + kC <= sp.len) {
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&bars[0], kTileB * (uint32_t)(nq + nk + nv + ndo));
+        const int z = (int)(sp.start + t0);
+        if (nq) tma_load_3d(tq, &tmq, &bars[0], 0, h, z);
+        if (nk) tma_load_3d(tk, &tmk, &bars[0], 0, h, z);
+        if (nv) tma_load_3d(tv, &tmv, &bars[0], 0, h, z);
+        if (ndo) tma_load_3d(tdo, &tmo, &bars[0], 0, h, z);
+      }
+      return true;
+    }
+    const int n = sp.len - t0;
+    const struct { bool need; const void* src; uint8_t* dst; } ts[4] = {
+        {nq, p.q, tq}, {nk, p.k, tk}, {nv, p.v, tv}, {ndo, p.dout, tdo}};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      if (!ts[x].need) continue;
+      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(ts[x].src);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int col = 32 * hf + 8 * jj;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (row < n) val = *reinterpret_cast<const uint4*>(src + row_of(t0 + row) * kD + col);
+        *reinterpret_cast<uint4*>(ts[x].dst + sw128_off(row, col)) = val;
+      }
+    }
+    fence_proxy_async_smem();
+    return false;
+  };
+
+  // Row `row`, columns 32*hf.., of a bf16 tile times f, split: hi in place, remainder in `lot`.
+  auto scale_split = [&](uint8_t* tile, uint8_t* lot, float f) {
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const uint32_t off = sw128_off(row, 32 * hf + 8 * jj);
+      const uint4 raw = *reinterpret_cast<const uint4*>(tile + off);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint32_t hi[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        split2(x.x * f, x.y * f, hi[e], lw[e]);
+      }
+      *reinterpret_cast<uint4*>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(lot + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+  };
+
+  const uint32_t qa = smem_u32(tq), ka = smem_u32(tk), va = smem_u32(tv), da = smem_u32(tdo);
+  const uint32_t qla = smem_u32(tqlo), kla = smem_u32(tklo);
+  const uint32_t sha = smem_u32(shi), sla = smem_u32(slo), uha = smem_u32(uhi), ula = smem_u32(ulo);
+  const int nt = (rend - lo + kC - 1) / kC;
+
+  // ---- pass 1: S = sum exp(g_m - g_s) k_s v_s^T (left), U = sum lam exp(g_t - g_m) q_t do_t^T ----
+  bool s_started = false, u_started = false;
+  for (int j = 0; j < nt; ++j) {
+    if (misc[1] != 0) break;
+    const int t0 = lo + j * kC;
+    const bool has_left = t0 < lend, has_right = t0 + kC > mid;
+    const bool tma = load(t0, has_right, has_left, has_left, has_right);
+    const int t = t0 + row;
+    float fS = 0.f, fU = 0.f;
+    if (has_left && t < lend) fS = expf((float)(gm - g[grow(t)]));
+    if (has_right && t >= mid && t < rend)
+      fU = p.lam[row_of(t) * p.L + lvl] * expf((float)(g[grow(t)] - gm));
+    if (tma) bwait(0, ph_ld);
+    if (has_left) scale_split(tk, tklo, fS);
+    if (has_right) scale_split(tq, tqlo, fU);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      if (misc[1] == 0) {
+        if (has_left) {
+#pragma unroll
+          for (int kk = 0; kk < kC / 16; ++kk)
+            mma_ss(tmem + kColS, mndesc(ka + kk * 2048), mndesc(va + kk * 2048), kIdescRed,
+                   (s_started || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kC / 16; ++kk)
+            mma_ss(tmem + kColS, mndesc(kla + kk * 2048), mndesc(va + kk * 2048), kIdescRed, 1u);
+        }
+        if (has_right) {
+#pragma unroll
+          for (int kk = 0; kk < kC / 16; ++kk)
+            mma_ss(tmem + kColU, mndesc(qa + kk * 2048), mndesc(da + kk * 2048), kIdescRed,
+                   (u_started || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kC / 16; ++kk)
+            mma_ss(tmem + kColU, mndesc(qla + kk * 2048), mndesc(da + kk * 2048), kIdescRed, 1u);
+        }
+      }
+      mma_commit(&bars[1]);
+    }
+    s_started = s_started || has_left;
+    u_started = u_started || has_right;
+    bwait(1, ph_mma);   // the tiles may be overwritten once the MMAs have read them
+    tc_fence_after();
+  }
+
+  // ---- S and U to shared memory, hi / lo (M = 64 accumulators: row i = 16 sub + lane) ----
+  if (misc[1] == 0) {
+    auto store_state = [&](uint8_t* dhi, uint8_t* dlo, const float (&x)[32]) {
+      const int i = 16 * sub + lane;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        uint32_t hi[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split2(x[8 * jj + 2 * e], x[8 * jj + 2 * e + 1], hi[e], lw[e]);
+        const uint32_t off = sw128_off(i, 32 * hf + 8 * jj);
+        *reinterpret_cast<uint4*>(dhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(dlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    };
+    float x[32];
+    tmem_ld32(tmem + lane_off + kColS + 32 * hf, x);
+    tmem_wait_ld();
+    if (lane < 16) store_state(shi, slo, x);
+    tmem_ld32(tmem + lane_off + kColU + 32 * hf, x);
+    tmem_wait_ld();
+    if (lane < 16) store_state(uhi, ulo, x);
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // ---- pass 2: W = dO S^T (right rows), DK = V U^T and DV = K U (left rows) ----
+  for (int j = 0; j < nt; ++j) {
+    if (misc[1] != 0) break;
+    const int t0 = lo + j * kC;
+    const bool has_left = t0 < lend, has_right = t0 + kC > mid;
+    const bool tma = load(t0, has_right, has_left, has_left, has_right);
+    if (tma) bwait(0, ph_ld);
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      if (misc[1] == 0) {
+        if (has_right) {
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss(tmem + kColW, kdesc(da + kk * 32), kdesc(sha + kk * 32), kIdescKK, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss(tmem + kColW, kdesc(da + kk * 32), kdesc(sla + kk * 32), kIdescKK, 1u);
+        }
+        if (has_left) {
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss(tmem + kColDK, kdesc(va + kk * 32), kdesc(uha + kk * 32), kIdescKK, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss(tmem + kColDK, kdesc(va + kk * 32), kdesc(ula + kk * 32), kIdescKK, 1u);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss(tmem + kColDV, kdesc(ka + kk * 32), mndesc(uha + kk * 2048), kIdescKN, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_ss(tmem + kColDV, kdesc(ka + kk * 32), mndesc(ula + kk * 2048), kIdescKN, 1u);
+        }
+      }
+      mma_commit(&bars[1]);
+    }
+    bwait(1, ph_mma);
+    tc_fence_after();
+    const int t = t0 + row;
+    const int wrow0 = t0 + 32 * sub;   // first token of this warp's rows
+    float dlp = 0.f;
+    const bool right_row = has_right && t >= mid && t < rend;
+    if (has_right && wrow0 + 31 >= mid) {   // warp-uniform: the TMEM load is .sync.aligned
+      float w[32];
+      tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
+      tmem_wait_ld();
+      if (right_row && misc[1] == 0) {
+        const size_t r = row_of(t);
+        const float sc = expf((float)(g[grow(t)] - gm));
+        const float lam = p.lam[r * p.L + lvl];
+        float* dq = p.dq + r * kD + 32 * hf;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float2 q01 = bf2_at(tq + sw128_off(row, 32 * hf + e));
+          const float2 q23 = bf2_at(tq + sw128_off(row, 32 * hf + e + 2));
+          const float w0 = sc * w[e], w1 = sc * w[e + 1], w2 = sc * w[e + 2], w3 = sc * w[e + 3];
+          dlp = fmaf(q01.x, w0, fmaf(q01.y, w1, fmaf(q23.x, w2, fmaf(q23.y, w3, dlp))));
+          float4 a = *reinterpret_cast<float4*>(dq + e);
+          a.x = fmaf(lam, w0, a.x);
+          a.y = fmaf(lam, w1, a.y);
+          a.z = fmaf(lam, w2, a.z);
+          a.w = fmaf(lam, w3, a.w);
+          *reinterpret_cast<float4*>(dq + e) = a;
+        }
+      }
+    }
+    if (has_left && wrow0 < lend) {
+      const bool left_row = t < lend && misc[1] == 0;
+      const size_t r = left_row ? row_of(t) : 0;
+      const float f = left_row ? expf((float)(gm - g[grow(t)])) : 0.f;
+      float x[32];
+      tmem_ld32(tmem + lane_off + kColDK + 32 * hf, x);
+      tmem_wait_ld();
+      if (left_row) {
+        float* dk = p.dk + r * kD + 32 * hf;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 a = *reinterpret_cast<float4*>(dk + e);
+          a.x = fmaf(f, x[e], a.x);
+          a.y = fmaf(f, x[e + 1], a.y);
+          a.z = fmaf(f, x[e + 2], a.z);
+          a.w = fmaf(f, x[e + 3], a.w);
+          *reinterpret_cast<float4*>(dk + e) = a;
+        }
+      }
+      tmem_ld32(tmem + lane_off + kColDV + 32 * hf, x);
+      tmem_wait_ld();
+      if (left_row) {
+        float* dv = p.dv + r * kD + 32 * hf;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 a = *reinterpret_cast<float4*>(dv + e);
+          a.x = fmaf(f, x[e], a.x);
+          a.y = fmaf(f, x[e + 1], a.y);
+          a.z = fmaf(f, x[e + 2], a.z);
+          a.w = fmaf(f, x[e + 3], a.w);
+          *reinterpret_cast<float4*>(dv + e) = a;
+        }
+      }
+    }
+    if (hf == 1) s_dl[row] = dlp;
+    __syncthreads();
+    if (hf == 0 && right_row && misc[1] == 0) p.dlam[row_of(t) * p.L + lvl] = dlp + s_dl[row];
+    tc_fence_before();
+    __syncthreads();   // TMEM drained and the tiles free for the next one
+  }
+
+  // a copy or MMA batch whose wait timed out must land before the CTA exits
+  if (stuck >= 0 && tid == 0) mbar_wait(&bars[stuck], stuck_par, 100000000ull);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool bwd_tc_supports(const BwdProblem& p) {
+  return p.in_dtype == LLATTN_BF16 && p.d == kD && p.L > kTcFirstLevel &&
+         (long long)p.nseq * p.T < (1ll << 31);
+}
+
+cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st) {
+  if (!bwd_tc_supports(p)) return cudaErrorNotSupported;
+  // TMA only fetches whole tiles inside a sequence, so for a packed batch any token extent
+  // >= the real total serves (nseq * T bounds it)
+  const long long tokens = (long long)p.nseq * p.T;
+  CUtensorMap mq, mk, mv, mo;
+  cudaError_t e;
+  if ((e = make_map(&mq, p.q, kD, p.H, tokens)) != cudaSuccess ||
+      (e = make_map(&mk, p.k, kD, p.H, tokens)) != cudaSuccess ||
+      (e = make_map(&mv, p.v, kD, p.H, tokens)) != cudaSuccess ||
+      (e = make_map(&mo, p.dout, kD, p.H, tokens)) != cudaSuccess)
+    return e;
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load()) {
+    if ((e = cudaFuncSetAttribute(bwd_level_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kSmemBytes)) != cudaSuccess)
+      return e;
+    attr_set[dev].store(true);
+  }
+  for (int lvl = kTcFirstLevel; lvl < p.L; ++lvl) {
+    const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
+    bwd_level_tc<<<dim3(nblk, p.H, p.nseq), kThreads, kSmemBytes, st>>>(mq, mk, mv, mo, p, g, lvl);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace llattn

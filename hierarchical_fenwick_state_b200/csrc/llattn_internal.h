@@ -1,6 +1,7 @@
 // Internal declarations shared by the host API and the kernel translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -41,6 +42,10 @@ bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T);
 void tc_set_segment_chunks(int chunks);
 int tc_segment_chunks(int nseq, int H, int T, int dk, int dv, bool varlen);
 bool tc_serial_supports(int in_dtype, int dk, int dv, int chunk, int T);
+
+// TMA map of a [tokens, H, rowlen] bf16 tensor viewed as {rowlen, H, tokens}: box {64, 1, 128}
+// (one 64-column slice of 128 rows), 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, int rowlen, int H, long long tokens);
 
 // Device address of the fixed scratch array behind llattn_fwd_noalloc on the
 // current device (looked up on the first call per device, then cached).

@@ -1569,6 +1569,8 @@ seg_blocks(int T, const int* __restrict__ cu, unsigned int* status, const SegArg
   }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -1577,7 +1579,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (fn == nullptr) {
     void* p = nullptr;
@@ -1604,6 +1606,8 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int rowlen, int H, long l
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+namespace {
 
 // out [tokens, H, rowlen] fp32 as {rowlen, H, tokens}; box {32, 1, 128} (128 B rows), 128 B swizzle.
 cudaError_t make_out_map(CUtensorMap* m, void* base, int rowlen, int H, long long tokens) {
