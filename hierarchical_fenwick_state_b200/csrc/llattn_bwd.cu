@@ -27,8 +27,8 @@
 // stay exact), the dense tiles (they initialise dq, dk, dv and dlam[:, 0..5]), one launch per
 // level 6..L-1 (each token sits in one block per level, so the updates of one launch never
 // collide), then dg per (token, head) and its reverse scan for dlog_a.  Arithmetic is fp32 on CUDA
-// cores, d = dk = dv in {32, 64, 128}; with bf16 inputs at d = 64 the levels from 7 on run on the
-// tensor cores instead (llattn_bwd_tc.cu).
+// cores, d = dk = dv in {32, 64, 128}; with bf16 inputs at d = 64 the pair interactions (dense
+// tiles and levels) run on the tensor cores instead (llattn_bwd_tc.cu).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -415,18 +415,20 @@ cudaError_t launch(const BwdProblem& p, double* g, cudaStream_t st) {
   }
   const dim3 seqs(p.H, p.nseq);
   bwd_prefix_g<<<seqs, 32, 0, st>>>(p, g);
-  bwd_dense_tile<Tin, D><<<dim3((p.T + kTile - 1) / kTile, p.H, p.nseq), kThreads,
-                           dense_smem_bytes<D>(), st>>>(p, g);
-  // levels from kTcFirstLevel on go to the tensor cores where they can (bf16, d = 64)
-  const bool tc = bwd_tc_supports(p);
-  const int lvl_end = tc ? kTcFirstLevel : p.L;
-  int n = 2;
-  for (int lvl = kDenseLevels; lvl < lvl_end; ++lvl, ++n) {
-    const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
-    bwd_level_block<Tin, D><<<dim3(nblk, p.H, p.nseq), kThreads, level_smem_bytes<D>(), st>>>(
-        p, g, lvl);
+  int n = 1;
+  if (bwd_tc_supports(p)) {
+    // bf16 at d = 64: every pair interaction on the tensor cores
+    if ((e = bwd_levels_tc(p, g, st)) != cudaSuccess) return e;
+  } else {
+    bwd_dense_tile<Tin, D><<<dim3((p.T + kTile - 1) / kTile, p.H, p.nseq), kThreads,
+                             dense_smem_bytes<D>(), st>>>(p, g);
+    ++n;
+    for (int lvl = kDenseLevels; lvl < p.L; ++lvl, ++n) {
+      const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
+      bwd_level_block<Tin, D><<<dim3(nblk, p.H, p.nseq), kThreads, level_smem_bytes<D>(), st>>>(
+          p, g, lvl);
+    }
   }
-  if (tc && (e = bwd_levels_tc(p, g, st)) != cudaSuccess) return e;
   bwd_dg<Tin, D><<<dim3((p.T + kThreads / 32 - 1) / (kThreads / 32), p.H, p.nseq), kThreads, 0,
                    st>>>(p);
   bwd_suffix_scan<<<seqs, kThreads, 0, st>>>(p);

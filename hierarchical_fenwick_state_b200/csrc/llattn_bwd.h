@@ -33,9 +33,11 @@ inline size_t bwd_workspace_bytes(int nseq, int H, int T) {
 
 cudaError_t bwd(const BwdProblem& p, void* ws, cudaStream_t st);
 
-// Levels kTcFirstLevel.. on the tensor cores (bf16 inputs, d = 64): one launch per level after
-// the dense tiles and the CUDA-core levels below it; g = the fp64 prefix sums of log_a.
-constexpr int kTcFirstLevel = 7;
+// The tensor-core backward (bf16 inputs, d = 64): one launch for the pairs inside each aligned
+// 128-token chunk (levels 0..7, the first write of every gradient), then one per level from
+// kTcFirstLevel on; g = the fp64 prefix sums of log_a.  In place of the dense tiles and the
+// CUDA-core level kernels.
+constexpr int kTcFirstLevel = 8;
 bool bwd_tc_supports(const BwdProblem& p);
 cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st);
 

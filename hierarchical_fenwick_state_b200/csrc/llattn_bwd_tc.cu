@@ -1,4 +1,5 @@
-// Backward pass, levels >= 7, on the tensor cores (bf16 inputs, d = 64).
+// Backward pass on the tensor cores (bf16 inputs, d = 64): the pairs inside each aligned chunk
+// of 128 tokens (levels 0..7), then one launch per level >= 8.
 //
 // Log-Linear Attention (gist.science summaries, Italian "Sommario tecnico" section 2, "Matrici
 // Gerarchiche"): at level l the positions fall into aligned blocks of 2^l tokens, and every key
@@ -12,7 +13,7 @@
 // for   w_t = exp(g_t - g_m) S do_t,  dlam[t, l] = q_t . w_t,  dq_t += lam[t, l] w_t,
 //       dk_s += exp(g_m - g_s) U v_s,  dv_s += exp(g_m - g_s) U^T k_s   (dlam = 0 on the left).
 //
-// One CTA takes one block and walks it twice in tiles of 128 tokens.  Pass 1 reduces S and U
+// Levels >= 8: one CTA takes one block and walks it twice in tiles of 128 tokens.  Pass 1 reduces S and U
 // over the tiles on the tensor cores (K^T V and Q^T dO shapes, M = 64, the token index as the
 // reduction dimension) into TMEM.  Pass 2 multiplies every tile by them: W = dO S^T,
 // DK = V U^T, DV = K U (M = 128 rows per tile), and the epilogue applies the exponential
@@ -412,11 +413,264 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   }
 }
 
+// ---- levels 0..7: the pairs inside one aligned chunk of 128 tokens ----
+//
+// With A = Q K^T, B = dO V^T and the chunk's mask M[t, s] = lam[t, l(t, s)] exp(g_t - g_s) for
+// s <= t (l <= 7 inside an aligned chunk):
+//   dQ = (M .* B) K,  dK = (M .* B)^T Q,  dV = (M .* A)^T dO,
+//   dlam[t, l] = sum over s with l(t, s) = l of exp(g_t - g_s) A[t, s] B[t, s].
+// One CTA per chunk: A and B on the tensor cores into TMEM, the masked products P1 = M .* B and
+// P2 = M .* A to shared memory (bf16 hi / lo, each as two 64-column halves in the 128-byte
+// swizzle), then the three products, which give this chunk's share of dq, dk and dv: the first
+// write of every gradient row (the levels >= 8 add to it).
+constexpr uint32_t kHalfB = kC * 128;                 // [128 rows][64 cols] bf16
+constexpr uint32_t kMatB = 2 * kHalfB;                // two halves: columns 0..63, 64..127
+constexpr uint32_t kIOffP1h = 4 * kTileB, kIOffP1l = kIOffP1h + kMatB;
+constexpr uint32_t kIOffP2h = kIOffP1l + kMatB, kIOffP2l = kIOffP2h + kMatB;
+constexpr uint32_t kIOffG = kIOffP2l + kMatB;         // g of the chunk's rows: [128] fp64
+constexpr uint32_t kIOffLam = kIOffG + kC * 8;        // lam[t, 0..7]: [128][9] fp32 (odd stride)
+constexpr uint32_t kIOffDl = kIOffLam + kC * 9 * 4;   // dlam partials of column half 1: [128][8]
+constexpr uint32_t kIOffBar = kIOffDl + kC * 8 * 4;
+constexpr uint32_t kIOffMisc = kIOffBar + 16;
+constexpr uint32_t kISmemBytes = kIOffMisc + 16 + 1024;
+static_assert(kISmemBytes <= 227 * 1024, "shared memory");
+
+constexpr uint32_t kIColA = 0, kIColB = 128, kIColDQ = 256, kIColDK = 320, kIColDV = 384;
+constexpr uint32_t kIdescAB = idesc_bf16(128, 128, 0, 0);   // rows x rows^T (both K-major)
+constexpr uint32_t kIdescTN = idesc_bf16(128, 64, 1, 1);    // P^T (M contiguous) x rows (N contiguous)
+
+// MN-major operand of M = 128 stored as two 64-element groups 16 KB apart (the halves).
+__device__ __forceinline__ uint64_t mndesc2(uint32_t saddr) { return sdesc_sw128(saddr, kHalfB, 1024); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+             const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+             const BwdProblem p, const double* __restrict__ g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int sub = warp & 3, hf = warp >> 2, row = sub * 32 + lane;
+  const uint32_t lane_off = uint32_t(sub * 32) << 16;
+  const int ch = blockIdx.x, h = blockIdx.y, sq = blockIdx.z;
+  const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
+  const int t0 = ch * kC;
+  if (t0 >= sp.len) return;
+  const int n = min(kC, sp.len - t0);
+  auto row_of = [&](int t) { return (size_t)(sp.start + t) * p.H + h; };
+
+  uint8_t* tq = sm + kOffQ;
+  uint8_t* tk = sm + kOffK;
+  uint8_t* tv = sm + kOffV;
+  uint8_t* tdo = sm + kOffDO;
+  uint8_t* p1h = sm + kIOffP1h;
+  uint8_t* p1l = sm + kIOffP1l;
+  uint8_t* p2h = sm + kIOffP2h;
+  uint8_t* p2l = sm + kIOffP2l;
+  double* s_g = reinterpret_cast<double*>(sm + kIOffG);
+  float* s_lam = reinterpret_cast<float*>(sm + kIOffLam);
+  float* s_dl = reinterpret_cast<float*>(sm + kIOffDl);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kIOffBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kIOffMisc);
+
+  if (warp == 0) {
+    tmem_alloc(&misc[0], 512);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+    misc[1] = 0;
+  }
+  // the chunk's tiles: TMA when the whole chunk lies inside the sequence, else plain loads
+  const bool tma = n == kC;
+  if (tma) {
+    if (tid == 32) {
+      mbar_arrive_expect_tx(&bars[0], 4 * kTileB);
+      const int z = (int)(sp.start + t0);
+      tma_load_3d(tq, &tmq, &bars[0], 0, h, z);
+      tma_load_3d(tk, &tmk, &bars[0], 0, h, z);
+      tma_load_3d(tv, &tmv, &bars[0], 0, h, z);
+      tma_load_3d(tdo, &tmo, &bars[0], 0, h, z);
+    }
+  } else {
+    const struct { const void* src; uint8_t* dst; } ts[4] = {
+        {p.q, tq}, {p.k, tk}, {p.v, tv}, {p.dout, tdo}};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(ts[x].src);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int col = 32 * hf + 8 * jj;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (row < n) val = *reinterpret_cast<const uint4*>(src + row_of(t0 + row) * kD + col);
+        *reinterpret_cast<uint4*>(ts[x].dst + sw128_off(row, col)) = val;
+      }
+    }
+    fence_proxy_async_smem();
+  }
+  // row scalars while the tiles fly
+  if (hf == 0) s_g[row] = row < n ? g[((size_t)sq * p.T + t0 + row) * p.H + h] : 0.0;
+  else {
+#pragma unroll
+    for (int l = 0; l < 8; ++l)
+      s_lam[row * 9 + l] = (row < n && l < p.L) ? p.lam[row_of(t0 + row) * p.L + l] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  uint32_t ph_mma = 0u;
+  int stuck = -1;
+  uint32_t stuck_par = 0u;
+  auto bwait = [&](int b, uint32_t ph) {
+    if (!mbar_wait(&bars[b], ph)) {
+      atomicOr(p.status, LLATTN_DEV_WAIT_TIMEOUT);
+      misc[1] = 1;
+      if (stuck < 0) {
+        stuck = b;
+        stuck_par = ph;
+      }
+    }
+  };
+  if (tma) bwait(0, 0u);
+  const uint32_t qa = smem_u32(tq), ka = smem_u32(tk), va = smem_u32(tv), da = smem_u32(tdo);
+
+  // ---- A = Q K^T, B = dO V^T ----
+  if (tid == 0) {
+    tc_fence_after();
+    if (misc[1] == 0) {
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_ss(tmem + kIColA, kdesc(qa + kk * 32), kdesc(ka + kk * 32), kIdescAB, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_ss(tmem + kIColB, kdesc(da + kk * 32), kdesc(va + kk * 32), kIdescAB, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&bars[1]);
+  }
+  bwait(1, ph_mma);
+  ph_mma ^= 1u;
+  tc_fence_after();
+
+  // ---- masks: P1 = M .* B, P2 = M .* A (hi / lo), and dlam's level sums ----
+  {
+    const int t = row;
+    const double gt = s_g[t];
+    const float* lr = s_lam + t * 9;
+    float dl[8];
+#pragma unroll
+    for (int l = 0; l < 8; ++l) dl[l] = 0.f;
+    const uint32_t hoff = hf * kHalfB;   // this thread's columns are half hf of each matrix
+#pragma unroll 1
+    for (int c16 = 0; c16 < 4; ++c16) {
+      const int s0 = 64 * hf + 16 * c16;
+      float av[16], bv[16];
+      tmem_ld16(tmem + lane_off + kIColA + s0, av);
+      tmem_ld16(tmem + lane_off + kIColB + s0, bv);
+      tmem_wait_ld();
+      float p1[16], p2[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int s = s0 + e;
+        float x1 = 0.f, x2 = 0.f;
+        if (s <= t && t < n) {
+          const float E = expf((float)(gt - s_g[s]));
+          const int lev = 32 - __clz(t ^ s);          // 0 when s == t
+          const float m = lr[lev] * E;
+          x1 = m * bv[e];
+          x2 = m * av[e];
+          const float xe = E * av[e] * bv[e];
+#pragma unroll
+          for (int l = 0; l < 8; ++l) dl[l] += l == lev ? xe : 0.f;
+        }
+        p1[e] = x1;
+        p2[e] = x2;
+      }
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
+        uint32_t h1[4], l1[4], h2[4], l2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          split2(p1[8 * hq + 2 * e], p1[8 * hq + 2 * e + 1], h1[e], l1[e]);
+          split2(p2[8 * hq + 2 * e], p2[8 * hq + 2 * e + 1], h2[e], l2[e]);
+        }
+        const uint32_t off = hoff + sw128_off(t, 16 * c16 + 8 * hq);
+        *reinterpret_cast<uint4*>(p1h + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+        *reinterpret_cast<uint4*>(p1l + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
+        *reinterpret_cast<uint4*>(p2h + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+        *reinterpret_cast<uint4*>(p2l + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
+      }
+    }
+    if (hf == 1) {
+#pragma unroll
+      for (int l = 0; l < 8; ++l) s_dl[t * 8 + l] = dl[l];
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (hf == 0 && t < n) {
+      float* dst = p.dlam + row_of(t0 + t) * p.L;
+#pragma unroll
+      for (int l = 0; l < 8; ++l)
+        if (l < p.L) dst[l] = dl[l] + s_dl[t * 8 + l];
+    }
+  }
+
+  // ---- dQ = P1 K, dK = P1^T Q, dV = P2^T dO (hi and lo parts) ----
+  if (tid == 0) {
+    tc_fence_after();
+    if (misc[1] == 0) {
+      const uint32_t a1h = smem_u32(p1h), a1l = smem_u32(p1l), a2h = smem_u32(p2h), a2l = smem_u32(p2l);
+#pragma unroll
+      for (int kk = 0; kk < kC / 16; ++kk) {
+        const uint32_t ko = (kk >> 2) * kHalfB + (kk & 3) * 32;   // K-major: half, then 16 keys
+        mma_ss(tmem + kIColDQ, kdesc(a1h + ko), mndesc(ka + kk * 2048), kIdescKN, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kIColDQ, kdesc(a1l + ko), mndesc(ka + kk * 2048), kIdescKN, 1u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kC / 16; ++kk) {
+        mma_ss(tmem + kIColDK, mndesc2(a1h + kk * 2048), mndesc(qa + kk * 2048), kIdescTN, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kIColDK, mndesc2(a1l + kk * 2048), mndesc(qa + kk * 2048), kIdescTN, 1u);
+        mma_ss(tmem + kIColDV, mndesc2(a2h + kk * 2048), mndesc(da + kk * 2048), kIdescTN, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kIColDV, mndesc2(a2l + kk * 2048), mndesc(da + kk * 2048), kIdescTN, 1u);
+      }
+    }
+    mma_commit(&bars[1]);
+  }
+  bwait(1, ph_mma);
+  ph_mma ^= 1u;
+  tc_fence_after();
+  {
+    const bool ok = row < n && misc[1] == 0;
+    const size_t r = ok ? row_of(t0 + row) * kD + 32 * hf : 0;
+    const struct { uint32_t col; float* dst; } outs[3] = {
+        {kIColDQ, p.dq}, {kIColDK, p.dk}, {kIColDV, p.dv}};
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      float v[32];
+      tmem_ld32(tmem + lane_off + outs[x].col + 32 * hf, v);
+      tmem_wait_ld();
+      if (ok) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(outs[x].dst + r + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      }
+    }
+  }
+  if (stuck >= 0 && tid == 0) mbar_wait(&bars[stuck], stuck_par, 100000000ull);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 bool bwd_tc_supports(const BwdProblem& p) {
-  return p.in_dtype == LLATTN_BF16 && p.d == kD && p.L > kTcFirstLevel &&
-         (long long)p.nseq * p.T < (1ll << 31);
+  return p.in_dtype == LLATTN_BF16 && p.d == kD && (long long)p.nseq * p.T < (1ll << 31);
 }
 
 cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st) {
@@ -437,10 +691,15 @@ cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st)
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev].load()) {
     if ((e = cudaFuncSetAttribute(bwd_level_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kSmemBytes)) != cudaSuccess)
+                                  (int)kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kISmemBytes)) != cudaSuccess)
       return e;
     attr_set[dev].store(true);
   }
+  // levels 0..7: one CTA per chunk, the first write of dq, dk, dv and dlam[:, 0..7]
+  bwd_intra_tc<<<dim3((p.T + kC - 1) / kC, p.H, p.nseq), kThreads, kISmemBytes, st>>>(mq, mk, mv, mo, p, g);
+  count_launch();
   for (int lvl = kTcFirstLevel; lvl < p.L; ++lvl) {
     const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
     bwd_level_tc<<<dim3(nblk, p.H, p.nseq), kThreads, kSmemBytes, st>>>(mq, mk, mv, mo, p, g, lvl);

@@ -384,10 +384,11 @@ LLATTN_API llattn_status llattn_prefill_state(int in_dtype, const void* k, const
  *
  * llattn_bwd
  *   in_dtype   LLATTN_BF16 or LLATTN_F32: the type of q, k, v and dout (bf16 as uint16 bit
- *              patterns).  Arithmetic is fp32 on CUDA cores, except that with bf16 inputs
- *              at d = 64 the block interactions of levels >= 7 (aligned blocks of >= 128
- *              tokens) run on the tensor cores, every derived operand split into bf16 high
- *              and low parts (fp32-accumulation accuracy).
+ *              patterns).  With bf16 inputs at d = 64 the pair interactions run on the
+ *              tensor cores (within each aligned 128-token chunk, then level by level over
+ *              larger aligned blocks), every derived operand split into bf16 high and low
+ *              parts (fp32-accumulation accuracy); otherwise arithmetic is fp32 on CUDA
+ *              cores.
  *   q, k, v, log_a, lam, B, H, T, cu_seqlens   as in llattn_fwd.
  *   dout       [B, T, H, dv] (packed: [total, H, dv]), the gradient of the loss at out.
  *   dq, dk, dv [.., H, d] fp32; dlog_a [.., H] fp32; dlam [.., H, L] fp32: fully overwritten

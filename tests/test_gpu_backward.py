@@ -6,8 +6,8 @@ ragged tail, one token, a packed batch with an empty and a one-token sequence, b
 and fp32 inputs, slow and the workloads' own decay.  At the benchmark's size (B=4,
 H=32, T=8192, d=64) sampled gradient rows and columns are compared with the oracle's
 direct sums.  The CUDA-core kernels compute in fp32 on the exact input values; the
-tensor-core levels (bf16, d = 64, levels >= 7) split every derived operand into bf16
-high and low parts, which keeps them at fp32-accumulation accuracy: the bound is 1e-4 of
+tensor-core kernels (bf16, d = 64) split every derived operand into bf16 high and low
+parts, which keeps them at fp32-accumulation accuracy: the bound is 1e-4 of
 each gradient's RMS for bf16 inputs too.
 """
 import numpy as np
