@@ -55,18 +55,23 @@ constexpr int kThreads = 256;    // warp w: TMEM lanes 32*(w%4).., column half w
 // ---- shared memory (bytes from a 1024-byte aligned base) ----
 constexpr uint32_t kTileB = kC * 128;            // 128 rows x 128 B, 128-byte swizzle
 constexpr uint32_t kOffQ = 0, kOffK = kTileB, kOffV = 2 * kTileB, kOffDO = 3 * kTileB;
-constexpr uint32_t kOffQlo = 4 * kTileB, kOffKlo = 5 * kTileB;
-constexpr uint32_t kState = kD * 128;            // 64 rows x 128 B
-constexpr uint32_t kOffShi = 6 * kTileB, kOffSlo = kOffShi + kState;
-constexpr uint32_t kOffUhi = kOffSlo + kState, kOffUlo = kOffUhi + kState;
-constexpr uint32_t kOffDl = kOffUlo + kState;    // dlam partials of column half 1: [128] fp32
-constexpr uint32_t kOffBar = kOffDl + kC * 4;    // [0] loads, [1] MMAs
-constexpr uint32_t kOffMisc = kOffBar + 16;      // [0] TMEM base, [1] abort
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 
-// ---- TMEM columns ----
-constexpr uint32_t kColS = 0, kColU = 64;        // M = 64 accumulators
-constexpr uint32_t kColW = 128, kColDK = 192, kColDV = 256;   // M = 128 accumulators
+// Level kernel: a tile lies in one half of its block (half >= 128 tokens), so it needs two
+// inputs: X = K, Y = V on the left, X = Q, Y = dO on the right.  About 81 KB and 128 TMEM
+// columns, so two CTAs share an SM and overlap their tile chains.
+constexpr uint32_t kState = kD * 128;            // 64 rows x 128 B
+constexpr uint32_t kLOffX = 0, kLOffY = kTileB, kLOffXlo = 2 * kTileB;
+constexpr uint32_t kLOffShi = 3 * kTileB, kLOffSlo = kLOffShi + kState;
+constexpr uint32_t kLOffUhi = kLOffSlo + kState, kLOffUlo = kLOffUhi + kState;
+constexpr uint32_t kLOffDl = kLOffUlo + kState;  // dlam partials of column half 1: [128] fp32
+constexpr uint32_t kLOffBar = kLOffDl + kC * 4;  // [0] loads, [1] MMAs
+constexpr uint32_t kLOffMisc = kLOffBar + 16;    // [0] TMEM base, [1] abort
+constexpr uint32_t kSmemBytes = kLOffMisc + 16 + 1024;
+
+// ---- TMEM columns of the level kernel (128 allocated) ----
+constexpr uint32_t kColS = 0, kColU = 64;        // pass 1: M = 64 accumulators
+constexpr uint32_t kColW = 0;                    // pass 2, right tiles: M = 128
+constexpr uint32_t kColDK = 0, kColDV = 64;      // pass 2, left tiles: M = 128
 
 constexpr uint32_t kIdescRed = idesc_bf16(64, 64, 1, 1);     // X^T (M contiguous) x Y (N contiguous)
 constexpr uint32_t kIdescKK = idesc_bf16(128, 64, 0, 0);     // rows (K-major) x state rows (K-major)
@@ -94,7 +99,7 @@ __device__ __forceinline__ float2 bf2_at(const uint8_t* p) {
 }
 
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
              const BwdProblem p, const double* __restrict__ g, int lvl) {
@@ -105,7 +110,7 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   const uint32_t lane_off = uint32_t(sub * 32) << 16;
   const int blk = blockIdx.x, h = blockIdx.y, sq = blockIdx.z;
   const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
-  const int half = 1 << (lvl - 1);
+  const int half = 1 << (lvl - 1);               // a multiple of 128 (lvl >= 8)
   const long long a0 = (long long)blk << lvl;
   if (a0 >= sp.len) return;
   const int lo = (int)a0, mid = lo + half;
@@ -116,22 +121,19 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   for (int t = lo + tid; t < lend; t += kThreads) p.dlam[row_of(t) * p.L + lvl] = 0.f;
   if (mid >= sp.len) return;   // no right half: nothing meets at this level
 
-  uint8_t* tq = sm + kOffQ;
-  uint8_t* tk = sm + kOffK;
-  uint8_t* tv = sm + kOffV;
-  uint8_t* tdo = sm + kOffDO;
-  uint8_t* tqlo = sm + kOffQlo;
-  uint8_t* tklo = sm + kOffKlo;
-  uint8_t* shi = sm + kOffShi;
-  uint8_t* slo = sm + kOffSlo;
-  uint8_t* uhi = sm + kOffUhi;
-  uint8_t* ulo = sm + kOffUlo;
-  float* s_dl = reinterpret_cast<float*>(sm + kOffDl);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
-  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+  uint8_t* tx = sm + kLOffX;
+  uint8_t* ty = sm + kLOffY;
+  uint8_t* txlo = sm + kLOffXlo;
+  uint8_t* shi = sm + kLOffShi;
+  uint8_t* slo = sm + kLOffSlo;
+  uint8_t* uhi = sm + kLOffUhi;
+  uint8_t* ulo = sm + kLOffUlo;
+  float* s_dl = reinterpret_cast<float*>(sm + kLOffDl);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kLOffBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kLOffMisc);
 
   if (warp == 0) {
-    tmem_alloc(&misc[0], 512);
+    tmem_alloc(&misc[0], 128);
     tmem_relinquish();
   }
   if (tid == 32) {
@@ -164,60 +166,38 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     ph ^= 1u;
   };
 
-  // One tile of 128 tokens from t0: the tensors a pass needs.  Whole tiles inside the sequence
-  // come by TMA (returns true: wait on bars[0]); a tile running past the sequence end by plain
-  // loads of its rows, the rest zero.
-  auto load = [&](int t0, bool nq, bool nk, bool nv, bool ndo) {
+  // The tile of 128 tokens from t0: X, Y = K, V (left) or Q, dO (right).  A whole tile inside
+  // the sequence comes by TMA (returns true: wait on bars[0]); a tile running past the sequence
+  // end by plain loads of its rows, the rest zero.
+  auto load = [&](int t0, bool left) {
     if (t0 + kC <= sp.len) {
       if (tid == 0) {
-        mbar_arrive_expect_tx(&bars[0], kTileB * (uint32_t)(nq + nk + nv + ndo));
+        mbar_arrive_expect_tx(&bars[0], 2 * kTileB);
         const int z = (int)(sp.start + t0);
-        if (nq) tma_load_3d(tq, &tmq, &bars[0], 0, h, z);
-        if (nk) tma_load_3d(tk, &tmk, &bars[0], 0, h, z);
-        if (nv) tma_load_3d(tv, &tmv, &bars[0], 0, h, z);
-        if (ndo) tma_load_3d(tdo, &tmo, &bars[0], 0, h, z);
+        tma_load_3d(tx, left ? &tmk : &tmq, &bars[0], 0, h, z);
+        tma_load_3d(ty, left ? &tmv : &tmo, &bars[0], 0, h, z);
       }
       return true;
     }
     const int n = sp.len - t0;
-    const struct { bool need; const void* src; uint8_t* dst; } ts[4] = {
-        {nq, p.q, tq}, {nk, p.k, tk}, {nv, p.v, tv}, {ndo, p.dout, tdo}};
+    const __nv_bfloat16* sx = static_cast<const __nv_bfloat16*>(left ? p.k : p.q);
+    const __nv_bfloat16* sy = static_cast<const __nv_bfloat16*>(left ? p.v : p.dout);
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      if (!ts[x].need) continue;
-      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(ts[x].src);
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int col = 32 * hf + 8 * jj;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (row < n) val = *reinterpret_cast<const uint4*>(src + row_of(t0 + row) * kD + col);
-        *reinterpret_cast<uint4*>(ts[x].dst + sw128_off(row, col)) = val;
+    for (int jj = 0; jj < 4; ++jj) {
+      const int col = 32 * hf + 8 * jj;
+      uint4 vx = make_uint4(0u, 0u, 0u, 0u), vy = vx;
+      if (row < n) {
+        vx = *reinterpret_cast<const uint4*>(sx + row_of(t0 + row) * kD + col);
+        vy = *reinterpret_cast<const uint4*>(sy + row_of(t0 + row) * kD + col);
       }
+      *reinterpret_cast<uint4*>(tx + sw128_off(row, col)) = vx;
+      *reinterpret_cast<uint4*>(ty + sw128_off(row, col)) = vy;
     }
     fence_proxy_async_smem();
     return false;
   };
 
-  // Row `row`, columns 32*hf.., of a bf16 tile times f, split: hi in place, remainder in `lot`.
-  auto scale_split = [&](uint8_t* tile, uint8_t* lot, float f) {
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const uint32_t off = sw128_off(row, 32 * hf + 8 * jj);
-      const uint4 raw = *reinterpret_cast<const uint4*>(tile + off);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-      uint32_t hi[4], lw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-        split2(x.x * f, x.y * f, hi[e], lw[e]);
-      }
-      *reinterpret_cast<uint4*>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(lot + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-  };
-
-  const uint32_t qa = smem_u32(tq), ka = smem_u32(tk), va = smem_u32(tv), da = smem_u32(tdo);
-  const uint32_t qla = smem_u32(tqlo), kla = smem_u32(tklo);
+  const uint32_t xa = smem_u32(tx), ya = smem_u32(ty), xla = smem_u32(txlo);
   const uint32_t sha = smem_u32(shi), sla = smem_u32(slo), uha = smem_u32(uhi), ula = smem_u32(ulo);
   const int nt = (rend - lo + kC - 1) / kC;
 
@@ -226,45 +206,51 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   for (int j = 0; j < nt; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
-    const bool has_left = t0 < lend, has_right = t0 + kC > mid;
-    const bool tma = load(t0, has_right, has_left, has_left, has_right);
+    const bool left = t0 < mid;
+    const bool tma = load(t0, left);
     const int t = t0 + row;
-    float fS = 0.f, fU = 0.f;
-    if (has_left && t < lend) fS = expf((float)(gm - g[grow(t)]));
-    if (has_right && t >= mid && t < rend)
-      fU = p.lam[row_of(t) * p.L + lvl] * expf((float)(g[grow(t)] - gm));
+    float f = 0.f;
+    if (left) {
+      if (t < lend) f = expf((float)(gm - g[grow(t)]));
+    } else if (t < rend) {
+      f = p.lam[row_of(t) * p.L + lvl] * expf((float)(g[grow(t)] - gm));
+    }
     if (tma) bwait(0, ph_ld);
-    if (has_left) scale_split(tk, tklo, fS);
-    if (has_right) scale_split(tq, tqlo, fU);
+    // X rows times f, split: hi in place, remainder in Xlo
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const uint32_t off = sw128_off(row, 32 * hf + 8 * jj);
+      const uint4 raw = *reinterpret_cast<const uint4*>(tx + off);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint32_t hi[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        split2(x.x * f, x.y * f, hi[e], lw[e]);
+      }
+      *reinterpret_cast<uint4*>(tx + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(txlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
       if (misc[1] == 0) {
-        if (has_left) {
+        const uint32_t d = tmem + (left ? kColS : kColU);
+        const bool started = left ? s_started : u_started;
 #pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
-            mma_ss(tmem + kColS, mndesc(ka + kk * 2048), mndesc(va + kk * 2048), kIdescRed,
-                   (s_started || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kC / 16; ++kk)
+          mma_ss(d, mndesc(xa + kk * 2048), mndesc(ya + kk * 2048), kIdescRed,
+                 (started || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
-            mma_ss(tmem + kColS, mndesc(kla + kk * 2048), mndesc(va + kk * 2048), kIdescRed, 1u);
-        }
-        if (has_right) {
-#pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
-            mma_ss(tmem + kColU, mndesc(qa + kk * 2048), mndesc(da + kk * 2048), kIdescRed,
-                   (u_started || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
-            mma_ss(tmem + kColU, mndesc(qla + kk * 2048), mndesc(da + kk * 2048), kIdescRed, 1u);
-        }
+        for (int kk = 0; kk < kC / 16; ++kk)
+          mma_ss(d, mndesc(xla + kk * 2048), mndesc(ya + kk * 2048), kIdescRed, 1u);
       }
       mma_commit(&bars[1]);
     }
-    s_started = s_started || has_left;
-    u_started = u_started || has_right;
+    s_started = s_started || left;
+    u_started = u_started || !left;
     bwait(1, ph_mma);   // the tiles may be overwritten once the MMAs have read them
     tc_fence_after();
   }
@@ -295,39 +281,38 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   tc_fence_before();
   __syncthreads();
 
-  // ---- pass 2: W = dO S^T (right rows), DK = V U^T and DV = K U (left rows) ----
+  // ---- pass 2: W = dO S^T (right tiles), DK = V U^T and DV = K U (left tiles) ----
   for (int j = 0; j < nt; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
-    const bool has_left = t0 < lend, has_right = t0 + kC > mid;
-    const bool tma = load(t0, has_right, has_left, has_left, has_right);
+    const bool left = t0 < mid;
+    const bool tma = load(t0, left);
     if (tma) bwait(0, ph_ld);
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
       if (misc[1] == 0) {
-        if (has_right) {
+        if (!left) {
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss(tmem + kColW, kdesc(da + kk * 32), kdesc(sha + kk * 32), kIdescKK, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + kColW, kdesc(ya + kk * 32), kdesc(sha + kk * 32), kIdescKK, kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss(tmem + kColW, kdesc(da + kk * 32), kdesc(sla + kk * 32), kIdescKK, 1u);
-        }
-        if (has_left) {
+            mma_ss(tmem + kColW, kdesc(ya + kk * 32), kdesc(sla + kk * 32), kIdescKK, 1u);
+        } else {
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss(tmem + kColDK, kdesc(va + kk * 32), kdesc(uha + kk * 32), kIdescKK, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + kColDK, kdesc(ya + kk * 32), kdesc(uha + kk * 32), kIdescKK, kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss(tmem + kColDK, kdesc(va + kk * 32), kdesc(ula + kk * 32), kIdescKK, 1u);
+            mma_ss(tmem + kColDK, kdesc(ya + kk * 32), kdesc(ula + kk * 32), kIdescKK, 1u);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss(tmem + kColDV, kdesc(ka + kk * 32), mndesc(uha + kk * 2048), kIdescKN, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + kColDV, kdesc(xa + kk * 32), mndesc(uha + kk * 2048), kIdescKN, kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk)
-            mma_ss(tmem + kColDV, kdesc(ka + kk * 32), mndesc(ula + kk * 2048), kIdescKN, 1u);
+            mma_ss(tmem + kColDV, kdesc(xa + kk * 32), mndesc(ula + kk * 2048), kIdescKN, 1u);
         }
       }
       mma_commit(&bars[1]);
@@ -335,10 +320,9 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     bwait(1, ph_mma);
     tc_fence_after();
     const int t = t0 + row;
-    const int wrow0 = t0 + 32 * sub;   // first token of this warp's rows
     float dlp = 0.f;
-    const bool right_row = has_right && t >= mid && t < rend;
-    if (has_right && wrow0 + 31 >= mid) {   // warp-uniform: the TMEM load is .sync.aligned
+    const bool right_row = !left && t < rend;
+    if (!left) {
       float w[32];
       tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
       tmem_wait_ld();
@@ -349,8 +333,8 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         float* dq = p.dq + r * kD + 32 * hf;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float2 q01 = bf2_at(tq + sw128_off(row, 32 * hf + e));
-          const float2 q23 = bf2_at(tq + sw128_off(row, 32 * hf + e + 2));
+          const float2 q01 = bf2_at(tx + sw128_off(row, 32 * hf + e));
+          const float2 q23 = bf2_at(tx + sw128_off(row, 32 * hf + e + 2));
           const float w0 = sc * w[e], w1 = sc * w[e + 1], w2 = sc * w[e + 2], w3 = sc * w[e + 3];
           dlp = fmaf(q01.x, w0, fmaf(q01.y, w1, fmaf(q23.x, w2, fmaf(q23.y, w3, dlp))));
           float4 a = *reinterpret_cast<float4*>(dq + e);
@@ -361,44 +345,35 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
           *reinterpret_cast<float4*>(dq + e) = a;
         }
       }
-    }
-    if (has_left && wrow0 < lend) {
+    } else {
       const bool left_row = t < lend && misc[1] == 0;
       const size_t r = left_row ? row_of(t) : 0;
       const float f = left_row ? expf((float)(gm - g[grow(t)])) : 0.f;
-      float x[32];
-      tmem_ld32(tmem + lane_off + kColDK + 32 * hf, x);
-      tmem_wait_ld();
-      if (left_row) {
-        float* dk = p.dk + r * kD + 32 * hf;
+      const struct { uint32_t col; float* dst; } outs[2] = {{kColDK, p.dk}, {kColDV, p.dv}};
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 a = *reinterpret_cast<float4*>(dk + e);
-          a.x = fmaf(f, x[e], a.x);
-          a.y = fmaf(f, x[e + 1], a.y);
-          a.z = fmaf(f, x[e + 2], a.z);
-          a.w = fmaf(f, x[e + 3], a.w);
-          *reinterpret_cast<float4*>(dk + e) = a;
-        }
-      }
-      tmem_ld32(tmem + lane_off + kColDV + 32 * hf, x);
-      tmem_wait_ld();
-      if (left_row) {
-        float* dv = p.dv + r * kD + 32 * hf;
+      for (int x = 0; x < 2; ++x) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + outs[x].col + 32 * hf, v);
+        tmem_wait_ld();
+        if (left_row) {
+          float* dst = outs[x].dst + r * kD + 32 * hf;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 a = *reinterpret_cast<float4*>(dv + e);
-          a.x = fmaf(f, x[e], a.x);
-          a.y = fmaf(f, x[e + 1], a.y);
-          a.z = fmaf(f, x[e + 2], a.z);
-          a.w = fmaf(f, x[e + 3], a.w);
-          *reinterpret_cast<float4*>(dv + e) = a;
+          for (int e = 0; e < 32; e += 4) {
+            float4 a = *reinterpret_cast<float4*>(dst + e);
+            a.x = fmaf(f, v[e], a.x);
+            a.y = fmaf(f, v[e + 1], a.y);
+            a.z = fmaf(f, v[e + 2], a.z);
+            a.w = fmaf(f, v[e + 3], a.w);
+            *reinterpret_cast<float4*>(dst + e) = a;
+          }
         }
       }
     }
-    if (hf == 1) s_dl[row] = dlp;
-    __syncthreads();
-    if (hf == 0 && right_row && misc[1] == 0) p.dlam[row_of(t) * p.L + lvl] = dlp + s_dl[row];
+    if (!left) {
+      if (hf == 1) s_dl[row] = dlp;
+      __syncthreads();
+      if (hf == 0 && right_row && misc[1] == 0) p.dlam[row_of(t) * p.L + lvl] = dlp + s_dl[row];
+    }
     tc_fence_before();
     __syncthreads();   // TMEM drained and the tiles free for the next one
   }
@@ -409,7 +384,7 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 128);
   }
 }
 
