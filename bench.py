@@ -134,6 +134,12 @@ def alu_peak_tflops():
     return 148 * 128 * 2 * 1.965e9 / 1e12
 
 
+def bwd_on_tensor_cores(inp):
+    """Whether llattn_bwd runs this problem's pair interactions on the tensor cores (bf16
+    inputs at d = 64), as the library dispatches it."""
+    return inp.dtype == "bf16" and inp.dk == 64 and inp.dv == 64
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -150,7 +156,8 @@ KERNEL_SOURCES = {
     "tcgen05": ["llattn_tc.cu", "llattn_tc_ptx.cuh", "llattn_common.cuh", "llattn_internal.h"],
     "simt": ["llattn_simt.cu", "llattn_common.cuh", "llattn_internal.h"],
     "decode": ["llattn_decode.cu", "llattn_decode.h", "llattn_common.cuh", "llattn_internal.h"],
-    "bwd": ["llattn_bwd.cu", "llattn_bwd.h", "llattn_common.cuh", "llattn_internal.h"],
+    "bwd": ["llattn_bwd.cu", "llattn_bwd.h", "llattn_bwd_tc.cu", "llattn_tc_ptx.cuh",
+            "llattn_common.cuh", "llattn_internal.h"],
 }
 
 
@@ -946,18 +953,27 @@ def run_bwd(args, w, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value = total_tokens * world / (ms_step / 1000.0)
 
-    hbm_gbs, _, peak_kind = measured_peaks()
+    hbm_gbs, bf16_tflops, peak_kind = measured_peaks()
     abytes, aflops, per_tok = bwd_algorithmic(w, lengths)
-    alu = alu_peak_tflops()
     main_avg_s = (main_ms / main_n) / 1000.0 if main_n else ms_step / 1000.0
     kernel_key = f"bwd:{w.name}"
-    if aflops / (alu * 1e12) >= abytes / (hbm_gbs * 1e9):
-        roof = {"bound": "alu", "achieved": aflops / main_avg_s / 1e12, "peak": alu,
-                "unit": "TFLOP/s",
-                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz (fp32 FMA)"}
+    peak_src = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "profiling-recipe fallback"
+    # bf16 at d = 64 runs every pair interaction on the tensor cores: its FLOPs count against
+    # the bf16 tensor peak; the other shapes compute in fp32 on CUDA cores
+    tensor = bwd_on_tensor_cores(inp)
+    if tensor:
+        cpeak, cunit, csrc = bf16_tflops, "TFLOP/s", peak_src + ", dense bf16 tensor"
+    else:
+        cpeak, cunit = alu_peak_tflops(), "TFLOP/s"
+        csrc = "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz (fp32 FMA)"
+    if aflops / (cpeak * 1e12) >= abytes / (hbm_gbs * 1e9):
+        roof = {"bound": "tensor" if tensor else "alu", "achieved": aflops / main_avg_s / 1e12,
+                "peak": cpeak, "unit": cunit, "peak_source": csrc}
     else:
         roof = {"bound": "hbm", "achieved": abytes / main_avg_s / 1e9, "peak": hbm_gbs,
-                "unit": "GB/s", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"}
+                "unit": "GB/s", "peak_source": peak_src}
+        roof["compute_frac"] = aflops / main_avg_s / 1e12 / cpeak
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = ncu_traffic(kernel_key)
     roof["kernel"] = kernel_key + " (all backward kernels of one call, one event pair)"
@@ -971,7 +987,8 @@ def run_bwd(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": bwd_config(w, "simt level-by-level"),
+        "config": bwd_config(w, "tensor cores: chunk pairs, then level by level" if tensor
+                             else "simt level-by-level"),
         "roofline": roof, "gpu_launches": launches, "clocks": clk,
     }
 

@@ -81,6 +81,7 @@ HEADLINE = "t8k_d64_bf16"
 PROFILE_WORKLOADS = {
     "t16k_d128_bf16_h8": Workload("t16k_d128_bf16_h8", B=1, H=8, T=16384, dk=128, dv=128,
                                   dtype="bf16", log_a_mu=-3.0),
+    "t8k_d64_bf16_b1": Workload("t8k_d64_bf16_b1", B=1, H=32, T=8192, dk=64, dv=64, dtype="bf16"),
 }
 
 # Log-Linear Gated DeltaNet forward: the same shapes and distributions (log_a is log alpha),
