@@ -739,6 +739,9 @@ tc_fwd_pipe(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUt
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // a later segment reads the pre-filled block states: the pre-pass must be complete (the first
+  // segment of a sequence starts while it still runs)
+  if (c0 > 0) griddep_wait();
   const uint32_t tmem = misc[0];
   auto W = [&](int b, uint32_t parity) { return pwait(&bars[b], parity, abort_flag, status); };
   auto is_full = [&](int c) { return (c0 + c + 1) * kC <= sp.len; };
@@ -1356,6 +1359,9 @@ tc_seg_total(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CU
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // seg_blocks may start now (it waits for this grid before it reads the totals), and with it
+  // the walk, whose first segments need no pre-fill
+  griddep_launch_dependents();
   const int h = blockIdx.x / sa.ndv, sq = blockIdx.y, J = blockIdx.z;
   const int vcol = (blockIdx.x % sa.ndv) * kD;
   const SeqSpan sp = seq_span(sq, T, cu, status);
@@ -1519,6 +1525,8 @@ seg_blocks(int T, const int* __restrict__ cu, unsigned int* status, const SegArg
            const float* __restrict__ seg_state, const float* __restrict__ seg_decay,
            uint8_t* __restrict__ blocks, float* __restrict__ block_decay) {
   extern __shared__ float cnt[];   // [levels][4096] fp32: the counter's slots
+  griddep_launch_dependents();     // the walk may start: its first segments need no pre-fill
+  griddep_wait();                  // the segment totals are complete
   const int t = threadIdx.x, sq = blockIdx.y;
   const SeqSpan sp = seq_span(sq, T, cu, status);
   const int nch_seq = (sp.len + kC - 1) / kC;
@@ -1717,14 +1725,33 @@ SegWorkspace seg_workspace(const SegPlan& pl, int nseq, int H, int dv, void* bas
   return w;
 }
 
+// A launch that may overlap the tail of the previous kernel in the stream (programmatic
+// dependent launch): used only after this library's own pre-pass kernels, which trigger it.
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  PdlLaunch(const dim3& grid, int threads, size_t smem, cudaStream_t st, bool pdl) {
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl ? 1 : 0;
+  }
+};
+
 template <typename LY, bool GEN>
-void launch_walk(const dim3& grid, cudaStream_t st, const CUtensorMap& mq, const CUtensorMap& mk,
-                 const CUtensorMap& mv, const CUtensorMap& mo, const Problem& p,
-                 const SegArgs& sa) {
-  tc_fwd_pipe<LY::kLev, LY::kSt, GEN><<<grid, kPThreads, LY::kSmemBytes, st>>>(
-      mq, mk, mv, mo, static_cast<const __nv_bfloat16*>(p.q),
-      static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v), p.log_a,
-      p.lam, p.out, p.H, p.T, p.L, p.cu_seqlens, p.status, sa);
+cudaError_t launch_walk(const dim3& grid, cudaStream_t st, const CUtensorMap& mq,
+                        const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                        const Problem& p, const SegArgs& sa, bool pdl) {
+  PdlLaunch l(grid, kPThreads, LY::kSmemBytes, st, pdl);
+  return cudaLaunchKernelEx(&l.cfg, tc_fwd_pipe<LY::kLev, LY::kSt, GEN>, mq, mk, mv, mo,
+                            static_cast<const __nv_bfloat16*>(p.q),
+                            static_cast<const __nv_bfloat16*>(p.k),
+                            static_cast<const __nv_bfloat16*>(p.v), p.log_a, p.lam, p.out, p.H,
+                            p.T, p.L, p.cu_seqlens, p.status, sa);
 }
 
 }  // namespace
@@ -1816,27 +1843,37 @@ cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, b
   for (int i = 0; i < p.dk / kD; ++i) {
     const SegArgs sa{pl.g, ndv, i * kD, p.dk, p.dv, i > 0 ? 1 : 0, w.blocks, w.block_decay,
                      pl.nblk, pl.nseg};
-    if (pl.nseg > 1) {
+    // Segments: the pre-pass (totals, then the counter over segments), then the walk.  The
+    // totals kernel waits for everything before it, as any launch; the counter and the walk
+    // are dependent launches that may start while their predecessor runs: the counter waits
+    // for the totals before it reads them, and only the walk's later segments wait for the
+    // counter (griddepcontrol), so the first segment of every sequence overlaps the pre-pass.
+    const bool pdl = pl.nseg > 1;
+    if (pdl) {
       tc_seg_total<<<dim3(vh, p.nseq, pl.nseg - 1), kSegThreads, kSegSmem, st>>>(
           mk, mv, p.log_a, p.H, p.T, p.cu_seqlens, p.status, sa, w.seg_state, w.seg_decay);
-      seg_blocks<<<dim3(vh, p.nseq), kBlkThreads, chunk_levels(pl.nseg) * kD * kD * sizeof(float),
-                   st>>>(p.T, p.cu_seqlens, p.status, sa, w.seg_state, w.seg_decay, w.blocks,
-                         w.block_decay);
+      PdlLaunch l(dim3(vh, p.nseq), kBlkThreads, chunk_levels(pl.nseg) * kD * kD * sizeof(float),
+                  st, true);
+      if ((e = cudaLaunchKernelEx(&l.cfg, seg_blocks, p.T, p.cu_seqlens, p.status, sa,
+                                  static_cast<const float*>(w.seg_state),
+                                  static_cast<const float*>(w.seg_decay), w.blocks,
+                                  w.block_decay)) != cudaSuccess)
+        break;
       count_launch(2);
     }
     const dim3 grid(vh, p.nseq, pl.nseg);
     const bool gen = pl.nseg > 1 || p.dk != kD || p.dv != kD;
     if (nch <= (1 << PipeShort::kLev)) {      // 6 levels on chip, three-stage ring
-      if (gen) launch_walk<PipeShort, true>(grid, st, mq, mk, mv, mo, p, sa);
-      else launch_walk<PipeShort, false>(grid, st, mq, mk, mv, mo, p, sa);
+      e = gen ? launch_walk<PipeShort, true>(grid, st, mq, mk, mv, mo, p, sa, pdl)
+              : launch_walk<PipeShort, false>(grid, st, mq, mk, mv, mo, p, sa, pdl);
     } else if (nch <= (1 << PipeLong::kLev)) {   // 7 levels, two stages (shared memory)
-      if (gen) launch_walk<PipeLong, true>(grid, st, mq, mk, mv, mo, p, sa);
-      else launch_walk<PipeLong, false>(grid, st, mq, mk, mv, mo, p, sa);
+      e = gen ? launch_walk<PipeLong, true>(grid, st, mq, mk, mv, mo, p, sa, pdl)
+              : launch_walk<PipeLong, false>(grid, st, mq, mk, mv, mo, p, sa, pdl);
     } else {                                  // 10 levels, two stages, always in segments
-      launch_walk<PipeXL, true>(grid, st, mq, mk, mv, mo, p, sa);
+      e = launch_walk<PipeXL, true>(grid, st, mq, mk, mv, mo, p, sa, pdl);
     }
     count_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) break;
+    if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) break;
   }
   main_kernel_end(st);
   return e == cudaSuccess ? cudaGetLastError() : e;
