@@ -36,7 +36,7 @@ namespace llattn {
 namespace {
 
 constexpr int kGdnWarps = 8;              // value columns per CTA
-constexpr int kGdnMaxLev = 17;            // levels held (T <= 65536)
+constexpr int kGdnMaxLev = 17;            // levels held at most (T <= 65536)
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -81,8 +81,8 @@ __device__ __forceinline__ void warp_sum16(float (&v)[16], int lane) {
 
 // Promotion: levels 0..m merge into level m + 1 and empty (m = trailing one bits of t).  A
 // switch on m (uniform over the warp) keeps every register index a constant.
-template <int R, int M>
-__device__ __forceinline__ void promote(float (&s)[kGdnMaxLev][R]) {
+template <int R, int NL, int M>
+__device__ __forceinline__ void promote(float (&s)[NL][R]) {
   float sum[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) sum[r] = 0.f;
@@ -97,29 +97,25 @@ __device__ __forceinline__ void promote(float (&s)[kGdnMaxLev][R]) {
   for (int r = 0; r < R; ++r) s[M + 1][r] = sum[r];
 }
 
-template <int R>
-__device__ __forceinline__ void promote_m(float (&s)[kGdnMaxLev][R], int m) {
+// m <= NL - 2 for positions t + 1 < 2^(NL - 1); the cases past that are never taken
+template <int R, int NL>
+__device__ __forceinline__ void promote_m(float (&s)[NL][R], int m) {
+#define LLATTN_GDN_PROMOTE(M) \
+  case M:                     \
+    if constexpr (M <= NL - 2) promote<R, NL, M>(s); \
+    break;
   switch (m) {
-    case 0: promote<R, 0>(s); break;
-    case 1: promote<R, 1>(s); break;
-    case 2: promote<R, 2>(s); break;
-    case 3: promote<R, 3>(s); break;
-    case 4: promote<R, 4>(s); break;
-    case 5: promote<R, 5>(s); break;
-    case 6: promote<R, 6>(s); break;
-    case 7: promote<R, 7>(s); break;
-    case 8: promote<R, 8>(s); break;
-    case 9: promote<R, 9>(s); break;
-    case 10: promote<R, 10>(s); break;
-    case 11: promote<R, 11>(s); break;
-    case 12: promote<R, 12>(s); break;
-    case 13: promote<R, 13>(s); break;
-    case 14: promote<R, 14>(s); break;
-    default: promote<R, 15>(s); break;   // m <= 15 for t < 65536
+    LLATTN_GDN_PROMOTE(0) LLATTN_GDN_PROMOTE(1) LLATTN_GDN_PROMOTE(2) LLATTN_GDN_PROMOTE(3)
+    LLATTN_GDN_PROMOTE(4) LLATTN_GDN_PROMOTE(5) LLATTN_GDN_PROMOTE(6) LLATTN_GDN_PROMOTE(7)
+    LLATTN_GDN_PROMOTE(8) LLATTN_GDN_PROMOTE(9) LLATTN_GDN_PROMOTE(10) LLATTN_GDN_PROMOTE(11)
+    LLATTN_GDN_PROMOTE(12) LLATTN_GDN_PROMOTE(13) LLATTN_GDN_PROMOTE(14) LLATTN_GDN_PROMOTE(15)
+    default: break;
   }
+#undef LLATTN_GDN_PROMOTE
 }
 
-template <typename TIn, int R>   // R = d_k / 32 rows of each column per lane
+// R = d_k / 32 rows of each column per lane; NL = levels held (sequences up to 2^(NL-1) tokens)
+template <typename TIn, int R, int NL>
 __global__ void __launch_bounds__(kGdnWarps * 32)
 gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                      const TIn* __restrict__ v, const float* __restrict__ log_alpha,
@@ -133,9 +129,10 @@ gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   const SeqSpan sp = seq_span(sq, T, cu, status);
   if (sp.len <= 0 || col >= dv) return;
 
-  float s[kGdnMaxLev][R];
+  static_assert(NL >= 2 && NL <= kGdnMaxLev, "the batched reduction takes up to 16 levels");
+  float s[NL][R];
 #pragma unroll
-  for (int l = 0; l < kGdnMaxLev; ++l)
+  for (int l = 0; l < NL; ++l)
 #pragma unroll
     for (int r = 0; r < R; ++r) s[l][r] = 0.f;
   uint32_t live = 0;   // bit l: level l holds a state (the binary counter of positions)
@@ -161,19 +158,20 @@ gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     float nk[R], nq[R], na = 0.f, nb = 0.f, nv = 0.f, nl = 0.f;
     if (t + 1 < sp.len) load(t + 1, nk, nq, na, nb, nv, nl);
     const float a = __expf(a_t), b = b_t;
-    // 1. transition of levels 1..16 (level 0 is rewritten below); empty levels stay zero
-    static_assert(kGdnMaxLev == 17, "the batched reduction takes 16 levels");
+    // 1. transition of levels 1..NL-1 (level 0 is rewritten below); empty levels stay zero
     {
       float p[16];
 #pragma unroll
-      for (int l = 1; l < kGdnMaxLev; ++l) {
+      for (int l = 1; l <= 16; ++l) {
         p[l - 1] = 0.f;
+        if (l < NL) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) p[l - 1] += kr[r] * s[l][r];
+          for (int r = 0; r < R; ++r) p[l - 1] += kr[r] * s[l][r];
+        }
       }
       warp_sum16(p, lane);
 #pragma unroll
-      for (int l = 1; l < kGdnMaxLev; ++l) {
+      for (int l = 1; l < NL; ++l) {
         const float pb = p[l - 1] * b;
 #pragma unroll
         for (int r = 0; r < R; ++r) s[l][r] = a * (s[l][r] - pb * kr[r]);
@@ -186,7 +184,7 @@ gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     // 3. readout: sum over occupied levels of lam[t, l] (q . s_l)
     float acc = 0.f;
 #pragma unroll
-    for (int l = 0; l < kGdnMaxLev; ++l) {
+    for (int l = 0; l < NL; ++l) {
       if (!((live >> l) & 1u)) continue;   // uniform over the warp; lam past L is never read
       const float wl = __shfl_sync(0xffffffffu, lam_t, l);
       float p = 0.f;
@@ -199,7 +197,7 @@ gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     // 4. promotion: levels 0..m into m + 1, m = trailing one bits of t
     if (t + 1 < sp.len) {
       const int m = __ffs(~t) - 1;
-      promote_m<R>(s, m);
+      promote_m<R, NL>(s, m);
       live = (live & ~((2u << m) - 1u)) | (1u << (m + 1));
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -214,25 +212,29 @@ gdn_recurrent_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   }
 }
 
+template <typename TIn, int R, int NL>
+void launch_r(const GdnProblem& p, const dim3& grid, cudaStream_t st) {
+  gdn_recurrent_kernel<TIn, R, NL><<<grid, kGdnWarps * 32, 0, st>>>(
+      static_cast<const TIn*>(p.q), static_cast<const TIn*>(p.k), static_cast<const TIn*>(p.v),
+      p.log_alpha, p.beta, p.lam, p.out, p.H, p.T, p.L, p.dv, p.cu_seqlens, p.status);
+}
+
+// Levels held: 12 for sequences up to 2048 tokens, 14 up to 8192, 17 up to 65536 (level l >= 1
+// is occupied only at positions t >= 2^(l-1)).
+template <typename TIn, int R>
+void launch_nl(const GdnProblem& p, const dim3& grid, cudaStream_t st) {
+  if (p.T <= 2048) launch_r<TIn, R, 12>(p, grid, st);
+  else if (p.T <= 8192) launch_r<TIn, R, 14>(p, grid, st);
+  else launch_r<TIn, R, kGdnMaxLev>(p, grid, st);
+}
+
 template <typename TIn>
 cudaError_t launch(const GdnProblem& p, cudaStream_t st) {
   const dim3 grid((p.dv + kGdnWarps - 1) / kGdnWarps, p.H, p.nseq);
-  const TIn* q = static_cast<const TIn*>(p.q);
-  const TIn* k = static_cast<const TIn*>(p.k);
-  const TIn* v = static_cast<const TIn*>(p.v);
   switch (p.dk) {
-    case 32:
-      gdn_recurrent_kernel<TIn, 1><<<grid, kGdnWarps * 32, 0, st>>>(
-          q, k, v, p.log_alpha, p.beta, p.lam, p.out, p.H, p.T, p.L, p.dv, p.cu_seqlens, p.status);
-      break;
-    case 64:
-      gdn_recurrent_kernel<TIn, 2><<<grid, kGdnWarps * 32, 0, st>>>(
-          q, k, v, p.log_alpha, p.beta, p.lam, p.out, p.H, p.T, p.L, p.dv, p.cu_seqlens, p.status);
-      break;
-    default:
-      gdn_recurrent_kernel<TIn, 4><<<grid, kGdnWarps * 32, 0, st>>>(
-          q, k, v, p.log_alpha, p.beta, p.lam, p.out, p.H, p.T, p.L, p.dv, p.cu_seqlens, p.status);
-      break;
+    case 32: launch_nl<TIn, 1>(p, grid, st); break;
+    case 64: launch_nl<TIn, 2>(p, grid, st); break;
+    default: launch_nl<TIn, 4>(p, grid, st); break;
   }
   return cudaGetLastError();
 }

@@ -48,6 +48,7 @@ CASES = {
     "t2k_d64_bf16": (I.shrink(W["t2k_d64_bf16"], B=1, H=2, T=2048), {}),
     "t256_d32_f32": (W["t256_d32_f32"], {}),
     "t700_d128_bf16": (I.shrink(W["t64k_d128_bf16"], H=2, T=700), {}),
+    "t2500_d32_f32": (I.Workload("gdn_t2500", B=1, H=2, T=2500, dk=32, dv=32, dtype="f32"), {}),
     "t500_beta1_slow": (I.shrink(W["t2k_d64_bf16"], B=1, H=3, T=500),
                         dict(beta_mode="ones", log_a_mode="slow")),
 }
@@ -90,5 +91,19 @@ def test_gdn_sampled_at_size():
     toks = np.concatenate([rng.integers(0, inp.total_tokens, 40), [0, 8191, 8192, 16383]])
     samples = [(int(t), int(h)) for t, h in zip(toks, rng.integers(0, inp.H, len(toks)))]
     ref = O.gdn_sampled(inp, samples)
+    err = O.rel_max_err(np.stack([got[t, h] for t, h in samples]), ref)
+    assert err <= TOL, f"sampled rel max err {err:.3e}"
+
+
+def test_gdn_deep_levels_long_sequence():
+    """T = 20000 runs the instantiation that holds 17 levels: level 15 (the bucket of the first
+    16384 tokens) alone weighs the output, sampled past position 16384."""
+    w = I.Workload("gdn_long", B=1, H=2, T=20000, dk=32, dv=32, dtype="bf16")
+    inp = I.make_gdn_inputs(w, seed=47, log_a_mode="slow", lam_mode="onehot", lam_level=15)
+    got = _run(inp).reshape(-1, inp.H, inp.dv)
+    assert np.isfinite(got).all()
+    samples = [(t, h) for t in (16384, 16385, 17001, 19999) for h in range(inp.H)]
+    ref = O.gdn_sampled(inp, samples)
+    assert np.abs(ref).max() > 0.0
     err = O.rel_max_err(np.stack([got[t, h] for t, h in samples]), ref)
     assert err <= TOL, f"sampled rel max err {err:.3e}"
