@@ -1844,16 +1844,18 @@ cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, b
     const SegArgs sa{pl.g, ndv, i * kD, p.dk, p.dv, i > 0 ? 1 : 0, w.blocks, w.block_decay,
                      pl.nblk, pl.nseg};
     // Segments: the pre-pass (totals, then the counter over segments), then the walk.  The
-    // totals kernel waits for everything before it, as any launch; the counter and the walk
-    // are dependent launches that may start while their predecessor runs: the counter waits
-    // for the totals before it reads them, and only the walk's later segments wait for the
-    // counter (griddepcontrol), so the first segment of every sequence overlaps the pre-pass.
-    const bool pdl = pl.nseg > 1;
-    if (pdl) {
+    // totals kernel waits for everything before it, as any launch.  Where its grid leaves SMs
+    // free, the counter and the walk are dependent launches that may start while their
+    // predecessor runs: the counter waits for the totals before it reads them, and only the
+    // walk's later segments wait for the counter (griddepcontrol), so the first segment of
+    // every sequence overlaps the pre-pass.  A pre-pass that fills the GPU gains nothing from
+    // it (measured 1-2% slower), so those launch in plain stream order.
+    const bool pdl = pl.nseg > 1 && (long long)vh * p.nseq * (pl.nseg - 1) < sm_count();
+    if (pl.nseg > 1) {
       tc_seg_total<<<dim3(vh, p.nseq, pl.nseg - 1), kSegThreads, kSegSmem, st>>>(
           mk, mv, p.log_a, p.H, p.T, p.cu_seqlens, p.status, sa, w.seg_state, w.seg_decay);
       PdlLaunch l(dim3(vh, p.nseq), kBlkThreads, chunk_levels(pl.nseg) * kD * kD * sizeof(float),
-                  st, true);
+                  st, pdl);
       if ((e = cudaLaunchKernelEx(&l.cfg, seg_blocks, p.T, p.cu_seqlens, p.status, sa,
                                   static_cast<const float*>(w.seg_state),
                                   static_cast<const float*>(w.seg_decay), w.blocks,
