@@ -540,27 +540,48 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
 #pragma unroll 1
     for (int c16 = 0; c16 < 4; ++c16) {
       const int s0 = 64 * hf + 16 * c16;
-      float av[16], bv[16];
-      tmem_ld16(tmem + lane_off + kIColA + s0, av);
-      tmem_ld16(tmem + lane_off + kIColB + s0, bv);
-      tmem_wait_ld();
       float p1[16], p2[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int s = s0 + e;
-        float x1 = 0.f, x2 = 0.f;
-        if (s <= t && t < n) {
-          const float E = expf((float)(gt - s_g[s]));
-          const int lev = 32 - __clz(t ^ s);          // 0 when s == t
-          const float m = lr[lev] * E;
-          x1 = m * bv[e];
-          x2 = m * av[e];
-          const float xe = E * av[e] * bv[e];
+      for (int e = 0; e < 16; ++e) p1[e] = p2[e] = 0.f;
+      if (s0 <= 32 * sub + 31) {   // warp-uniform: some row of this warp reaches these keys
+        float av[16], bv[16];
+        tmem_ld16(tmem + lane_off + kIColA + s0, av);
+        tmem_ld16(tmem + lane_off + kIColB + s0, bv);
+        tmem_wait_ld();
+        if (t < n && s0 <= t) {
+          if ((t >> 4) != (s0 >> 4)) {
+            // every key of the group is earlier, at one level: 1 + msb(t ^ s), fixed by bits >= 4
+            const int lev = 32 - __clz(t ^ s0);
+            const float lam = lr[lev];
+            float xs = 0.f;
 #pragma unroll
-          for (int l = 0; l < 8; ++l) dl[l] += l == lev ? xe : 0.f;
+            for (int e = 0; e < 16; ++e) {
+              const float E = expf((float)(gt - s_g[s0 + e]));
+              const float m = lam * E;
+              p1[e] = m * bv[e];
+              p2[e] = m * av[e];
+              xs = fmaf(E * av[e], bv[e], xs);
+            }
+#pragma unroll
+            for (int l = 0; l < 8; ++l) dl[l] += l == lev ? xs : 0.f;
+          } else {
+            // the row's own 16-key block: levels 0..4 element by element, keys s <= t only
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int s = s0 + e;
+              if (s <= t) {
+                const float E = expf((float)(gt - s_g[s]));
+                const int lev = 32 - __clz(t ^ s);   // 0 when s == t
+                const float m = lr[lev] * E;
+                p1[e] = m * bv[e];
+                p2[e] = m * av[e];
+                const float xe = E * av[e] * bv[e];
+#pragma unroll
+                for (int l = 0; l < 5; ++l) dl[l] += l == lev ? xe : 0.f;
+              }
+            }
+          }
         }
-        p1[e] = x1;
-        p2[e] = x2;
       }
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
