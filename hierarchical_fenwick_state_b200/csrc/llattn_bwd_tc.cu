@@ -317,55 +317,71 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       }
       mma_commit(&bars[1]);
     }
+    // the gradient row this thread adds to is read while the MMAs run (dq on the right, dk on
+    // the left; dv after the first drain, to stay inside the register budget)
+    const int t = t0 + row;
+    const bool right_row = !left && t < rend;
+    const bool left_row = left && t < lend;
+    const size_t r = (right_row || left_row) ? row_of(t) : 0;
+    float* dst0 = (left ? p.dk : p.dq) + r * kD + 32 * hf;
+    float4 old0[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      old0[e] = (right_row || left_row) ? *reinterpret_cast<const float4*>(dst0 + 4 * e)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
     bwait(1, ph_mma);
     tc_fence_after();
-    const int t = t0 + row;
     float dlp = 0.f;
-    const bool right_row = !left && t < rend;
     if (!left) {
       float w[32];
       tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
       tmem_wait_ld();
       if (right_row && misc[1] == 0) {
-        const size_t r = row_of(t);
         const float sc = expf((float)(g[grow(t)] - gm));
         const float lam = p.lam[r * p.L + lvl];
-        float* dq = p.dq + r * kD + 32 * hf;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float2 q01 = bf2_at(tx + sw128_off(row, 32 * hf + e));
           const float2 q23 = bf2_at(tx + sw128_off(row, 32 * hf + e + 2));
           const float w0 = sc * w[e], w1 = sc * w[e + 1], w2 = sc * w[e + 2], w3 = sc * w[e + 3];
           dlp = fmaf(q01.x, w0, fmaf(q01.y, w1, fmaf(q23.x, w2, fmaf(q23.y, w3, dlp))));
-          float4 a = *reinterpret_cast<float4*>(dq + e);
+          float4 a = old0[e / 4];
           a.x = fmaf(lam, w0, a.x);
           a.y = fmaf(lam, w1, a.y);
           a.z = fmaf(lam, w2, a.z);
           a.w = fmaf(lam, w3, a.w);
-          *reinterpret_cast<float4*>(dq + e) = a;
+          *reinterpret_cast<float4*>(dst0 + e) = a;
         }
       }
     } else {
-      const bool left_row = t < lend && misc[1] == 0;
-      const size_t r = left_row ? row_of(t) : 0;
-      const float f = left_row ? expf((float)(gm - g[grow(t)])) : 0.f;
-      const struct { uint32_t col; float* dst; } outs[2] = {{kColDK, p.dk}, {kColDV, p.dv}};
+      const bool ok = left_row && misc[1] == 0;
+      const float f = ok ? expf((float)(gm - g[grow(t)])) : 0.f;
+      float v[32];
+      tmem_ld32(tmem + lane_off + kColDK + 32 * hf, v);
+      tmem_wait_ld();
+      if (ok) {
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + outs[x].col + 32 * hf, v);
-        tmem_wait_ld();
-        if (left_row) {
-          float* dst = outs[x].dst + r * kD + 32 * hf;
+        for (int e = 0; e < 32; e += 4) {
+          float4 a = old0[e / 4];
+          a.x = fmaf(f, v[e], a.x);
+          a.y = fmaf(f, v[e + 1], a.y);
+          a.z = fmaf(f, v[e + 2], a.z);
+          a.w = fmaf(f, v[e + 3], a.w);
+          *reinterpret_cast<float4*>(dst0 + e) = a;
+        }
+      }
+      tmem_ld32(tmem + lane_off + kColDV + 32 * hf, v);
+      tmem_wait_ld();
+      if (ok) {
+        float* dv = p.dv + r * kD + 32 * hf;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 a = *reinterpret_cast<float4*>(dst + e);
-            a.x = fmaf(f, v[e], a.x);
-            a.y = fmaf(f, v[e + 1], a.y);
-            a.z = fmaf(f, v[e + 2], a.z);
-            a.w = fmaf(f, v[e + 3], a.w);
-            *reinterpret_cast<float4*>(dst + e) = a;
-          }
+        for (int e = 0; e < 32; e += 4) {
+          float4 a = *reinterpret_cast<float4*>(dv + e);
+          a.x = fmaf(f, v[e], a.x);
+          a.y = fmaf(f, v[e + 1], a.y);
+          a.z = fmaf(f, v[e + 2], a.z);
+          a.w = fmaf(f, v[e + 3], a.w);
+          *reinterpret_cast<float4*>(dv + e) = a;
         }
       }
     }
