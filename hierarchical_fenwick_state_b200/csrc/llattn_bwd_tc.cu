@@ -203,17 +203,34 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
 
   // ---- pass 1: S = sum exp(g_m - g_s) k_s v_s^T (left), U = sum lam exp(g_t - g_m) q_t do_t^T ----
   bool s_started = false, u_started = false;
+  // this row's prefix sum (and lam on the right) of tile j, read one tile ahead
+  auto row_in = [&](int j, double& gt, float& lt) {
+    const int t = lo + j * kC + row;
+    const bool left = lo + j * kC < mid;
+    gt = 0.0;
+    lt = 0.f;
+    if (j < nt && t < (left ? lend : rend)) {
+      gt = g[grow(t)];
+      if (!left) lt = p.lam[row_of(t) * p.L + lvl];
+    }
+  };
+  double g_next;
+  float l_next;
+  row_in(0, g_next, l_next);
   for (int j = 0; j < nt; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
     const bool left = t0 < mid;
     const bool tma = load(t0, left);
     const int t = t0 + row;
+    const double gt = g_next;
+    const float lt = l_next;
+    row_in(j + 1, g_next, l_next);
     float f = 0.f;
     if (left) {
-      if (t < lend) f = expf((float)(gm - g[grow(t)]));
+      if (t < lend) f = expf((float)(gm - gt));
     } else if (t < rend) {
-      f = p.lam[row_of(t) * p.L + lvl] * expf((float)(g[grow(t)] - gm));
+      f = lt * expf((float)(gt - gm));
     }
     if (tma) bwait(0, ph_ld);
     // X rows times f, split: hi in place, remainder in Xlo
@@ -329,6 +346,8 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     for (int e = 0; e < 8; ++e)
       old0[e] = (right_row || left_row) ? *reinterpret_cast<const float4*>(dst0 + 4 * e)
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    const double gt = (right_row || left_row) ? g[grow(t)] : gm;
+    const float lam = right_row ? p.lam[r * p.L + lvl] : 0.f;
     bwait(1, ph_mma);
     tc_fence_after();
     float dlp = 0.f;
@@ -337,8 +356,7 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
       tmem_wait_ld();
       if (right_row && misc[1] == 0) {
-        const float sc = expf((float)(g[grow(t)] - gm));
-        const float lam = p.lam[r * p.L + lvl];
+        const float sc = expf((float)(gt - gm));
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float2 q01 = bf2_at(tx + sw128_off(row, 32 * hf + e));
@@ -355,7 +373,7 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       }
     } else {
       const bool ok = left_row && misc[1] == 0;
-      const float f = ok ? expf((float)(gm - g[grow(t)])) : 0.f;
+      const float f = ok ? expf((float)(gm - gt)) : 0.f;
       float v[32];
       tmem_ld32(tmem + lane_off + kColDK + 32 * hf, v);
       tmem_wait_ld();
