@@ -49,23 +49,32 @@ constexpr int kTile = 32;        // dense tile: levels 0..5
 constexpr int kDenseLevels = 6;
 constexpr int kThreads = 256;
 
-// ---- g: inclusive prefix sums of log_a per (sequence, head), one warp each ----
-__global__ void bwd_prefix_g(BwdProblem p, double* g) {
-  const int h = blockIdx.x, sq = blockIdx.y, lane = threadIdx.x;
+// ---- g: inclusive prefix sums of log_a per (sequence, head), one CTA each ----
+// Each thread sums a contiguous segment of the sequence, a block scan of the segment totals
+// gives every segment its offset, and the thread writes its segment's prefix sums (fp64).
+__global__ void __launch_bounds__(kThreads) bwd_prefix_g(BwdProblem p, double* g) {
+  __shared__ double s_part[kThreads];
+  const int h = blockIdx.x, sq = blockIdx.y, tid = threadIdx.x;
   const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
-  double carry = 0.0;
-  for (int base = 0; base < sp.len; base += 32) {
-    const int t = base + lane;
-    const size_t row = (size_t)(sp.start + t) * p.H + h;
-    double x = t < sp.len ? (double)p.log_a[row] : 0.0;   // row is read only for t < len
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const double y = __shfl_up_sync(kFull, x, off);
-      if (lane >= off) x += y;
-    }
-    x += carry;
-    if (t < sp.len) g[((size_t)sq * p.T + t) * p.H + h] = x;
-    carry = __shfl_sync(kFull, x, 31);
+  const int seg = (sp.len + kThreads - 1) / kThreads;
+  const int t0 = min(tid * seg, sp.len), t1 = min(t0 + seg, sp.len);
+  const float* la = p.log_a + (size_t)sp.start * p.H + h;   // token t at la[t * H]
+  double* gg = g + (size_t)sq * p.T * p.H + h;              // local position t at gg[t * H]
+  double sum = 0.0;
+  for (int t = t0; t < t1; ++t) sum += (double)la[(size_t)t * p.H];
+  s_part[tid] = sum;
+  __syncthreads();
+  // inclusive prefix sums of the per-thread totals (Hillis-Steele)
+  for (int off = 1; off < kThreads; off <<= 1) {
+    const double y = tid >= off ? s_part[tid - off] : 0.0;
+    __syncthreads();
+    s_part[tid] += y;
+    __syncthreads();
+  }
+  double run = tid > 0 ? s_part[tid - 1] : 0.0;   // everything before this segment
+  for (int t = t0; t < t1; ++t) {
+    run += (double)la[(size_t)t * p.H];
+    gg[(size_t)t * p.H] = run;
   }
 }
 
@@ -414,7 +423,7 @@ cudaError_t launch(const BwdProblem& p, double* g, cudaStream_t st) {
     attr_set[dev].store(true);
   }
   const dim3 seqs(p.H, p.nseq);
-  bwd_prefix_g<<<seqs, 32, 0, st>>>(p, g);
+  bwd_prefix_g<<<seqs, kThreads, 0, st>>>(p, g);
   int n = 1;
   if (bwd_tc_supports(p)) {
     // bf16 at d = 64: every pair interaction on the tensor cores
