@@ -60,8 +60,20 @@ __global__ void __launch_bounds__(kThreads) bwd_prefix_g(BwdProblem p, double* g
   const int t0 = min(tid * seg, sp.len), t1 = min(t0 + seg, sp.len);
   const float* la = p.log_a + (size_t)sp.start * p.H + h;   // token t at la[t * H]
   double* gg = g + (size_t)sq * p.T * p.H + h;              // local position t at gg[t * H]
+  // segments of up to 32 tokens (T <= 8192) stay in registers between the two walks
+  constexpr int kReg = 32;
+  const bool in_reg = seg <= kReg;
+  float xr[kReg];
   double sum = 0.0;
-  for (int t = t0; t < t1; ++t) sum += (double)la[(size_t)t * p.H];
+  if (in_reg) {
+#pragma unroll
+    for (int i = 0; i < kReg; ++i) {
+      xr[i] = t0 + i < t1 ? la[(size_t)(t0 + i) * p.H] : 0.f;
+      sum += (double)xr[i];
+    }
+  } else {
+    for (int t = t0; t < t1; ++t) sum += (double)la[(size_t)t * p.H];
+  }
   s_part[tid] = sum;
   __syncthreads();
   // inclusive prefix sums of the per-thread totals (Hillis-Steele)
@@ -72,9 +84,17 @@ __global__ void __launch_bounds__(kThreads) bwd_prefix_g(BwdProblem p, double* g
     __syncthreads();
   }
   double run = tid > 0 ? s_part[tid - 1] : 0.0;   // everything before this segment
-  for (int t = t0; t < t1; ++t) {
-    run += (double)la[(size_t)t * p.H];
-    gg[(size_t)t * p.H] = run;
+  if (in_reg) {
+#pragma unroll
+    for (int i = 0; i < kReg; ++i) {
+      run += (double)xr[i];
+      if (t0 + i < t1) gg[(size_t)(t0 + i) * p.H] = run;
+    }
+  } else {
+    for (int t = t0; t < t1; ++t) {
+      run += (double)la[(size_t)t * p.H];
+      gg[(size_t)t * p.H] = run;
+    }
   }
 }
 
@@ -388,8 +408,20 @@ __global__ void __launch_bounds__(kThreads) bwd_suffix_scan(BwdProblem p) {
   const int seg = (sp.len + kThreads - 1) / kThreads;
   const int t0 = min(tid * seg, sp.len), t1 = min(t0 + seg, sp.len);
   float* x = p.dlog_a + (size_t)sp.start * p.H + h;   // token t at x[t * H]
+  // segments of up to 32 tokens (T <= 8192) stay in registers between the two walks
+  constexpr int kReg = 32;
+  const bool in_reg = seg <= kReg;
+  float xr[kReg];
   double sum = 0.0;
-  for (int t = t0; t < t1; ++t) sum += x[(size_t)t * p.H];
+  if (in_reg) {
+#pragma unroll
+    for (int i = 0; i < kReg; ++i) {
+      xr[i] = t0 + i < t1 ? x[(size_t)(t0 + i) * p.H] : 0.f;
+      sum += xr[i];
+    }
+  } else {
+    for (int t = t0; t < t1; ++t) sum += x[(size_t)t * p.H];
+  }
   s_part[tid] = sum;
   __syncthreads();
   // suffix sums of the per-thread totals (Hillis-Steele, reading the later entries)
@@ -400,9 +432,17 @@ __global__ void __launch_bounds__(kThreads) bwd_suffix_scan(BwdProblem p) {
     __syncthreads();
   }
   double run = tid + 1 < kThreads ? s_part[tid + 1] : 0.0;  // everything after this segment
-  for (int t = t1 - 1; t >= t0; --t) {
-    run += x[(size_t)t * p.H];
-    x[(size_t)t * p.H] = (float)run;
+  if (in_reg) {
+#pragma unroll
+    for (int i = kReg - 1; i >= 0; --i) {
+      run += xr[i];
+      if (t0 + i < t1) x[(size_t)(t0 + i) * p.H] = (float)run;
+    }
+  } else {
+    for (int t = t1 - 1; t >= t0; --t) {
+      run += x[(size_t)t * p.H];
+      x[(size_t)t * p.H] = (float)run;
+    }
   }
 }
 
