@@ -320,9 +320,10 @@ class OraclePool:
         self.pool.close()
         self.pool.join()
 
-    def rate(self, inp):
-        """Every head of the first sequence, spread over the cores; returns (tok/s of the
-        whole workload, cores used, description, wall seconds)."""
+    def rate(self, inp, heads=None, tokens=None):
+        """`heads` heads (default: all) of the first sequence, its first `tokens` tokens
+        (default: all), spread over the cores, one head per task; returns (tok/s of the whole
+        workload, cores used, description, wall seconds)."""
         import numpy as np
         start, n = inp.seq_slices()[0]
         sl = slice(start, start + n)
@@ -337,15 +338,19 @@ class OraclePool:
 
         # every worker started (imports done) before the clock: a tiny task each
         self.pool.map(_oracle_head_worker, [head(0, min(n, 8))] * self.cores)
-        work = [head(h) for h in range(inp.H)]
-        used = min(self.cores, inp.H)
+        nh = inp.H if heads is None else max(1, min(heads, inp.H))
+        m = n if tokens is None else max(1, min(tokens, n))
+        work = [head(h, m) for h in range(nh)]
+        used = min(self.cores, nh)
         t0 = time.perf_counter()
         self.pool.map(_oracle_head_worker, work, chunksize=1)
         wall = time.perf_counter() - t0
-        desc = (f"recurrent fp64 oracle form, 1 sequence x all {inp.H} heads x {n} tokens, one "
+        which = f"all {inp.H}" if nh == inp.H else f"{nh} of {inp.H}"
+        desc = (f"recurrent fp64 oracle form, 1 sequence x {which} heads x {m} tokens, one "
                 f"head per task on {used} host cores (spawned pool, single-threaded BLAS each), "
                 f"{wall:.2f} s wall")
-        return n / wall, used, desc, wall
+        # tokens/s of the whole workload: the sample is m tokens x nh / H of the heads
+        return m * nh / inp.H / wall, used, desc, wall
 
 
 def oracle_allcores_rate(inp):
@@ -384,12 +389,15 @@ def run_reference(args, w, rank, world):
         return None
     inp = I.make_inputs(w, seed=args.seed)
     pool = OraclePool()
+    # one round of the pool per step: as many heads of the first sequence as there are cores,
+    # so the default run (100 steps) stays within a few minutes; warm-up steps on a short sample
+    heads = min(inp.H, pool.cores)
     try:
         for _ in range(args.warmup):
-            oracle_sample_rate(inp, 1)
+            pool.rate(inp, heads=heads, tokens=256)
         times, rates = [], []
         for _ in range(args.steps):
-            r, cores, desc, dt = pool.rate(inp)
+            r, cores, desc, dt = pool.rate(inp, heads=heads)
             times.append(dt)
             rates.append(r)
     finally:
