@@ -137,8 +137,13 @@ llattn_status forward(int in_dtype, int path, int chunk, const void* q, const vo
   if (B < 0 || H < 0 || T < 0) return LLATTN_ERR_SHAPE;
   if (!head_dim_ok(dk) || !head_dim_ok(dv)) return LLATTN_ERR_SHAPE;
   if (T > (1 << 24) || H > 65535 || B > 65535) return LLATTN_ERR_SHAPE;
+  // the automatic choice with the default chunk takes the one-launch CUDA-core kernel for short
+  // sequences where the tensor cores do not apply (a path or chunk the caller names is kept)
+  const bool auto_default = path == LLATTN_PATH_AUTO && chunk == 0;
   llattn_status s = resolve(in_dtype, &path, &chunk, T, dk, dv);
   if (s != LLATTN_OK) return s;
+  const bool short_path = auto_default && path == LLATTN_PATH_SIMT &&
+                          llattn::simt_short_supports(T, llattn_num_levels(T));
   if (B == 0 || H == 0 || T == 0) return LLATTN_OK;  // nothing to compute
   if (!q || !k || !v || !log_a || !lam || !out) return LLATTN_ERR_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
@@ -166,14 +171,16 @@ llattn_status forward(int in_dtype, int path, int chunk, const void* q, const vo
   DeviceState* ds = nullptr;
   int dev = 0;
   if ((s = device_state(&ds, &dev)) != LLATTN_OK) return s;
-  const size_t need = workspace_for(path, chunk, B, H, T, dk, dv, cu_seqlens != nullptr);
+  const size_t need =
+      short_path ? 0 : workspace_for(path, chunk, B, H, T, dk, dv, cu_seqlens != nullptr);
   void* ws = workspace;
   std::unique_lock<std::mutex> lock(g_mu, std::defer_lock);
   if ((s = pick_workspace(ds, need, workspace, workspace_bytes, lock, &ws)) != LLATTN_OK) return s;
   llattn::Problem p{in_dtype, q, k, v, log_a, lam, out, B, H, T, dk, dv, L, cu_seqlens,
                     ds->status};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = path == LLATTN_PATH_SIMT
+  cudaError_t e = short_path ? llattn::simt_short_forward(p, st)
+                  : path == LLATTN_PATH_SIMT
                       ? llattn::simt_forward(p, chunk, ws, st)
                       : llattn::tc_forward(p, chunk, ws, st, path == LLATTN_PATH_TCGEN05_SERIAL);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -312,7 +319,7 @@ llattn_status llattn_fwd_bf16(const void* q, const void* k, const void* v, const
 llattn_status llattn_fwd_f32(const float* q, const float* k, const float* v, const float* log_a,
                              const float* lam, float* out, int B, int H, int T, int dk, int dv,
                              const int* cu_seqlens, void* stream) {
-  return forward(LLATTN_F32, LLATTN_PATH_SIMT, 0, q, k, v, log_a, lam, out, B, H, T, dk, dv,
+  return forward(LLATTN_F32, LLATTN_PATH_AUTO, 0, q, k, v, log_a, lam, out, B, H, T, dk, dv,
                  cu_seqlens, nullptr, 0, stream);
 }
 

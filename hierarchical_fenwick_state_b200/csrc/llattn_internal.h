@@ -35,6 +35,9 @@ size_t tc_workspace_bytes(int nseq, int H, int T, int dk, int dv, int chunk, boo
 
 // Kernel launchers; return a cudaError_t from the launches.
 cudaError_t simt_forward(const Problem& p, int chunk, void* ws, cudaStream_t st);
+// Short sequences on CUDA cores in one launch (the masked form; T <= 512).
+bool simt_short_supports(int T, int L);
+cudaError_t simt_short_forward(const Problem& p, cudaStream_t st);
 cudaError_t tc_forward(const Problem& p, int chunk, void* ws, cudaStream_t st, bool serial);
 bool tc_supports(int in_dtype, int dk, int dv, int chunk, int T);
 // Segment length of the tensor-core path: the forced value (chunks, 0 = automatic), and the

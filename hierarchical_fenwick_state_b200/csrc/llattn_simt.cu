@@ -15,8 +15,11 @@
 //                          states that queries read (one per even block index)
 //   3. simt_intra_readout  intra-chunk masked part plus the lam-weighted readout
 //                          of the block states, written to out (fp32)
+// Sequences of at most 512 tokens can instead take simt_short_fwd (below), the masked form in
+// one launch.
 // This path is the fp32-input product path (it keeps fp32 accuracy end to end)
 // and a cross-check for the tensor-core path on bf16 inputs.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -26,6 +29,8 @@
 
 namespace llattn {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int kThreads = 256;
 constexpr int kMaxLevels = 32;
@@ -286,6 +291,223 @@ cudaError_t launch_all(const Problem& p, int C, void* ws, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------------
+// Short sequences (T <= 512): the masked quadratic form itself ("Matrici Gerarchiche": out =
+// ((Q K^T) .* M_H) V), one launch.  At this size a whole sequence's keys fit a few shared-memory
+// tiles, and the three chunkwise launches cost more than the arithmetic.
+// A row block is 16 query rows of a (sequence, head), 16 threads per row.  Those 16 split the
+// columns into CL interleaved slices (CL = max(dk, dv) / 32, so a slice holds at most 32
+// columns) and the keys of each tile into KL = 16 / CL strided subsets: a thread forms the q.k
+// dot product of its keys over its column slice (reduced over the CL slices by shuffles), and
+// accumulates its keys' weighted v into its own slice of the output row.  The KL partial rows
+// are summed by shuffles at the end.  Keys arrive in shared-memory tiles of 32 rows (16 for
+// max(dk, dv) = 128), the next tile read into registers while the current one is used; a row is
+// padded by CL floats, so the 16 lanes of a row read 16 different banks.
+// Each thread reads a whole k and v row from shared memory per key, so a row block's cost is
+// its shared-memory reads.  When the grid is small, a thread-block cluster of KS CTAs (2 or 4)
+// shares one row block: rank r takes the key tiles r, r + KS, ..., and rank 0 adds the ranks'
+// partial rows in rank order through distributed shared memory.
+// The prefix sums g stay fp64 in shared memory, so the decay exp(g_t - g_s) is a difference of
+// exact values.
+// ---------------------------------------------------------------------------------------------
+constexpr int kShortMaxT = 512;
+constexpr int kShortRows = 16;
+constexpr int kShortLanes = kThreads / kShortRows;   // 16 threads per query row
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kThreads)
+simt_short_fwd(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+               const float* __restrict__ log_a, const float* __restrict__ lam,
+               float* __restrict__ out, int H, int T, int L, int KS, const int* __restrict__ cu,
+               unsigned int* status) {
+  constexpr int CL = (DK > DV ? DK : DV) / 32;      // column slices: 1, 2 or 4
+  constexpr int KL = kShortLanes / CL;              // key subsets: 16, 8 or 4
+  constexpr int TILE = CL == 4 ? 16 : 32;           // keys per tile
+  constexpr int SK = DK / CL, SV = DV / CL;         // columns of this thread's slices
+  constexpr int PK = DK + CL, PV = DV + CL;         // padded shared-memory rows
+  constexpr int FK = TILE * DK / kThreads;          // tile elements each thread fetches
+  constexpr int FV = TILE * DV / kThreads;
+  static_assert(CL * KL == kShortLanes && FK >= 1 && FV >= 1 && TILE % KL == 0, "short split");
+  __shared__ double s_g[kShortMaxT];
+  __shared__ float s_k[TILE * PK], s_v[TILE * PV];
+  __shared__ float s_lam[kShortRows][kMaxLevels / 2 + 1];
+  __shared__ float s_o[kShortRows * DV];            // this CTA's partial rows
+  const int rank = KS > 1 ? (int)(blockIdx.x % KS) : 0;
+  const int rb = blockIdx.x / KS, h = blockIdx.y, sq = blockIdx.z, tid = threadIdx.x;
+  const SeqSpan sp = seq_span(sq, T, cu, status);
+  const int r0 = rb * kShortRows;
+  if (r0 >= sp.len) return;                     // the whole cluster leaves together
+  const int n = min(r0 + kShortRows, sp.len);   // keys 0 .. n-1 reach the rows r0 .. n-1
+  auto row = [&](int t) { return (size_t)(sp.start + t) * H + h; };
+
+  // a key tile into registers (element e of the tile is row e / D, column e % D)
+  float fk[FK], fv[FV];
+  auto fetch = [&](int k0) {
+    const int m = min(TILE, n - k0);
+#pragma unroll
+    for (int u = 0; u < FK; ++u) {
+      const int e = tid + u * kThreads, i = e / DK;
+      fk[u] = i < m ? ld_in(k + row(k0 + i) * DK + (e % DK)) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < FV; ++u) {
+      const int e = tid + u * kThreads, i = e / DV;
+      fv[u] = i < m ? ld_in(v + row(k0 + i) * DV + (e % DV)) : 0.f;
+    }
+  };
+  const int kfirst = rank * TILE, kstep = KS * TILE;
+  if (kfirst < n) fetch(kfirst);
+
+  // this thread's query row and column slice, and the row block's lam (loads in flight together
+  // with the first key tile and log a)
+  const int r = tid / kShortLanes, j = tid % kShortLanes, t = r0 + r;
+  const int cl = j % CL, kl = j / CL;
+  const bool row_ok = t < n;
+  for (int e = tid; e < kShortRows * L; e += kThreads) {
+    const int rr = e / L, l = e % L;
+    s_lam[rr][l] = r0 + rr < n ? __ldg(lam + row(r0 + rr) * L + l) : 0.f;
+  }
+  float qs[SK];
+#pragma unroll
+  for (int e = 0; e < SK; ++e) qs[e] = row_ok ? ld_in(q + row(t) * DK + cl + CL * e) : 0.f;
+
+  // prefix sums of log a over positions 0 .. n-1: per-thread pairs, a warp scan, a block carry
+  {
+    const int i0 = 2 * tid;
+    const double a = i0 < n ? (double)__ldg(log_a + row(i0)) : 0.0;
+    const double b = i0 + 1 < n ? (double)__ldg(log_a + row(i0 + 1)) : 0.0;
+    double x = a + b;
+    const int lane = tid & 31, w = tid >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    __shared__ double s_w[kThreads / 32];
+    if (lane == 31) s_w[w] = x;
+    __syncthreads();
+    double off = 0.0;
+    for (int u = 0; u < w; ++u) off += s_w[u];
+    x += off;                                   // inclusive sum through position i0 + 1
+    if (i0 < n) s_g[i0] = x - b;
+    if (i0 + 1 < n) s_g[i0 + 1] = x;
+  }
+  float acc[SV];
+#pragma unroll
+  for (int e = 0; e < SV; ++e) acc[e] = 0.f;
+  __syncthreads();
+  const double gt = row_ok ? s_g[t] : 0.0;
+
+  for (int k0 = kfirst; k0 < n; k0 += kstep) {
+    __syncthreads();   // the previous tile is consumed
+#pragma unroll
+    for (int u = 0; u < FK; ++u) {
+      const int e = tid + u * kThreads;
+      s_k[(e / DK) * PK + e % DK] = fk[u];
+    }
+#pragma unroll
+    for (int u = 0; u < FV; ++u) {
+      const int e = tid + u * kThreads;
+      s_v[(e / DV) * PV + e % DV] = fv[u];
+    }
+    __syncthreads();
+    if (k0 + kstep < n) fetch(k0 + kstep);
+#pragma unroll
+    for (int ii = 0; ii < TILE / KL; ++ii) {
+      const int i = kl + KL * ii, s = k0 + i;
+      const float* kr = s_k + i * PK + cl;
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < SK; e += 2) {
+        d0 = fmaf(qs[e], kr[CL * e], d0);
+        if (e + 1 < SK) d1 = fmaf(qs[e + 1], kr[CL * (e + 1)], d1);
+      }
+      float d = d0 + d1;
+#pragma unroll
+      for (int o = 1; o < CL; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      if (row_ok && s <= t) {
+        const int lev = s == t ? 0 : 32 - __clz(t ^ s);
+        const float wgt = s_lam[r][lev] * expf((float)(gt - s_g[s])) * d;
+        const float* vr = s_v + i * PV + cl;
+#pragma unroll
+        for (int e = 0; e < SV; ++e) acc[e] = fmaf(wgt, vr[CL * e], acc[e]);
+      }
+    }
+  }
+  // the KL partial rows of a query row (lanes kl * CL + cl), summed over kl
+#pragma unroll
+  for (int o = CL; o < kShortLanes; o <<= 1) {
+#pragma unroll
+    for (int e = 0; e < SV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  }
+  if (KS == 1) {
+    if (row_ok && kl == 0) {
+      float* o = out + row(t) * DV + cl;
+#pragma unroll
+      for (int e = 0; e < SV; ++e) o[CL * e] = acc[e];
+    }
+    return;
+  }
+  if (kl == 0) {
+#pragma unroll
+    for (int e = 0; e < SV; ++e) s_o[r * DV + cl + CL * e] = acc[e];
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();                                   // every rank's partial rows are written
+  if (rank == 0) {
+    for (int e = tid; e < (n - r0) * DV; e += kThreads) {
+      float x = s_o[e];
+      for (int src = 1; src < KS; ++src) x += cluster.map_shared_rank(s_o, src)[e];
+      out[row(r0 + e / DV) * DV + e % DV] = x;
+    }
+  }
+  cluster.sync();                                   // rank 0 has read them
+}
+
+template <typename Tin, int DK>
+void launch_short_dk(const Problem& p, const cudaLaunchConfig_t& cfg, int KS) {
+  const Tin* q = static_cast<const Tin*>(p.q);
+  const Tin* k = static_cast<const Tin*>(p.k);
+  const Tin* v = static_cast<const Tin*>(p.v);
+  switch (p.dv) {
+    case 32: cudaLaunchKernelEx(&cfg, simt_short_fwd<Tin, DK, 32>, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, KS, p.cu_seqlens, p.status); break;
+    case 64: cudaLaunchKernelEx(&cfg, simt_short_fwd<Tin, DK, 64>, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, KS, p.cu_seqlens, p.status); break;
+    default: cudaLaunchKernelEx(&cfg, simt_short_fwd<Tin, DK, 128>, q, k, v, p.log_a, p.lam, p.out, p.H, p.T, p.L, KS, p.cu_seqlens, p.status); break;
+  }
+}
+
+// Cluster size of the short form: 4 CTAs per row block while the row blocks alone fill at most
+// half the SMs, 2 while they fill at most all of them, else 1.
+int short_split(long long row_blocks) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  return 2 * row_blocks <= sms ? 4 : row_blocks <= sms ? 2 : 1;
+}
+
+template <typename Tin>
+void launch_short(const Problem& p, cudaStream_t st) {
+  const int nrb = (p.T + kShortRows - 1) / kShortRows;
+  const int KS = short_split((long long)nrb * p.H * p.nseq);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nrb * KS, p.H, p.nseq);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = KS > 1 ? 1 : 0;
+  switch (p.dk) {
+    case 32: launch_short_dk<Tin, 32>(p, cfg, KS); break;
+    case 64: launch_short_dk<Tin, 64>(p, cfg, KS); break;
+    default: launch_short_dk<Tin, 128>(p, cfg, KS); break;
+  }
+}
+
 }  // namespace
 
 size_t simt_workspace_bytes(int nseq, int H, int T, int dk, int dv, int C) {
@@ -300,6 +522,18 @@ size_t simt_workspace_bytes(int nseq, int H, int T, int dk, int dv, int C) {
 cudaError_t simt_forward(const Problem& p, int C, void* ws, cudaStream_t st) {
   if (p.in_dtype == LLATTN_BF16) return launch_all<__nv_bfloat16>(p, C, ws, st);
   return launch_all<float>(p, C, ws, st);
+}
+
+bool simt_short_supports(int T, int L) { return T <= kShortMaxT && L <= kMaxLevels / 2 + 1; }
+
+cudaError_t simt_short_forward(const Problem& p, cudaStream_t st) {
+  if (!simt_short_supports(p.T, p.L)) return cudaErrorNotSupported;
+  main_kernel_begin(st);
+  if (p.in_dtype == LLATTN_BF16) launch_short<__nv_bfloat16>(p, st);
+  else launch_short<float>(p, st);
+  main_kernel_end(st);
+  count_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace llattn

@@ -77,7 +77,11 @@ typedef enum {
 enum { LLATTN_F32 = 0, LLATTN_BF16 = 1 };
 
 /* Kernel paths for llattn_fwd_ex.
- *   AUTO            tcgen05 path where one exists for the shape, else SIMT.
+ *   AUTO            tcgen05 path where one exists for the shape, else SIMT.  With chunk 0, a
+ *                   call that resolves to SIMT with T <= 512 runs the masked (quadratic) form
+ *                   in one launch instead of the chunkwise kernels: at that length the whole
+ *                   key range of a query fits a few shared-memory tiles.  It needs no
+ *                   workspace and computes in fp32 like SIMT.
  *   SIMT            CUDA-core kernels (any dk, dv in {32,64,128}; fp32 or bf16 inputs).
  *   TCGEN05         tensor-core kernel, warp-specialised pipeline (bf16 inputs, d_k and
  *                   d_v in {64, 128}, chunk 128, T <= 131072; the serial cross-check d = 64,
@@ -136,7 +140,8 @@ LLATTN_API llattn_status llattn_fwd_bf16(const void* q, const void* k, const voi
                                          void* stream);
 
 /* llattn_fwd_f32 - the same operation on fp32 q, k, v (CUDA-core fp32 path, no
- * tensor cores, so results meet a 1e-4 relative bound).  Arguments as llattn_fwd. */
+ * tensor cores, so results meet a 1e-4 relative bound; the automatic path, so T <= 512 runs
+ * the one-launch masked form).  Arguments as llattn_fwd. */
 LLATTN_API llattn_status llattn_fwd_f32(const float* q, const float* k, const float* v, const float* log_a,
                              const float* lam, float* out, int B, int H, int T, int dk, int dv,
                              const int* cu_seqlens, void* stream);

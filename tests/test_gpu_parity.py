@@ -277,6 +277,23 @@ def test_fwd_bf16_alias_matches_fwd():
     assert binding.stream_status(clear=True) == 0
 
 
+
+@pytest.mark.parametrize("T", [300, 700])
+def test_fwd_f32_entry_both_sides_of_the_short_form(T):
+    """llattn_fwd_f32 takes the automatic path: T = 300 runs the one-launch masked form, T = 700
+    the chunkwise CUDA-core kernels; both against the oracle at the fp32 bound."""
+    import torch
+    w = I.Workload("f32_entry", B=2, H=3, T=T, dk=64, dv=32, dtype="f32")
+    inp = I.make_inputs(w, seed=T)
+    t = _to_device_for_guard(inp)
+    out = torch.full(inp.v.shape, float("nan"), dtype=torch.float32, device="cuda:0")
+    binding.fwd_f32(t["q"], t["k"], t["v"], t["log_a"], t["lam"], out, inp.B, inp.H, inp.T,
+                    inp.dk, inp.dv)
+    torch.cuda.synchronize()
+    assert binding.stream_status(clear=True) == 0
+    err = O.rel_max_err(out.double().cpu().numpy(), O.llattn_recurrent(inp))
+    assert err <= TOL["f32"], f"rel max err {err:.3e}"
+
 # ------------------------------------------------------------------------------------------------
 # Segments: a CTA walks 2^g chunks, the levels above its segment pre-filled from the block
 # states the pre-pass builds (segment totals on the tensor cores, then the counter over segments)
@@ -346,3 +363,43 @@ def test_long_context_d128_deep_levels():
     ref = O.llattn_recurrent(inp)
     assert binding.segment_plan(inp.B, inp.H, inp.T, inp.dk, inp.dv) > 0
     _check(inp, ref, "tcgen05")
+
+
+# ------------------------------------------------------------------------------------------------
+# Short sequences through the automatic path: the one-launch masked form on CUDA cores
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("T,dk,dv,dtype,mode", [
+    (256, 32, 32, "f32", "dist"),
+    (1, 32, 32, "f32", "dist"),
+    (33, 64, 64, "f32", "slow"),
+    (500, 128, 64, "f32", "strong"),
+    (512, 64, 32, "f32", "zero"),
+    (300, 32, 128, "bf16", "dist"),
+    (129, 32, 32, "bf16", "slow"),
+])
+def test_short_sequences_one_launch(T, dk, dv, dtype, mode):
+    """T <= 512 where the tensor cores do not apply (fp32, or d_k = 32): the automatic path
+    with the default chunk runs the masked form in one launch; every output element against the
+    oracle, the last 16-row block ragged where T is not a multiple of 16.  With 2 x 3 heads the
+    row blocks number 6 * ceil(T / 16): T <= 192 splits each block's keys over a cluster of 4
+    CTAs, T = 256 and 300 over 2, and T = 500 and 512 run one CTA per block."""
+    w = I.Workload("short", B=2, H=3, T=T, dk=dk, dv=dv, dtype=dtype)
+    inp = I.make_inputs(w, seed=T + dk + dv, log_a_mode=mode)
+    ref = O.llattn_quadratic(inp)
+    _check(inp, ref, "auto")
+
+
+def test_short_sequences_packed_one_launch():
+    lengths = np.array([0, 1, 100, 512, 37, 64])
+    w = I.Workload("short_vl", B=len(lengths), H=2, T=512, dk=32, dv=32, dtype="f32", varlen=True)
+    inp = I.make_inputs(w, seed=71, lengths=lengths)
+    _check(inp, O.llattn_quadratic(inp), "auto")
+
+
+def test_short_sequences_packed_cluster_split():
+    """Few row blocks (4 sequences of at most 128 tokens, 2 heads): the keys of a block are
+    split over a cluster of 4 CTAs, including blocks with fewer key tiles than CTAs."""
+    lengths = np.array([0, 1, 100, 37, 128])
+    w = I.Workload("short_vl4", B=len(lengths), H=2, T=128, dk=64, dv=64, dtype="f32", varlen=True)
+    inp = I.make_inputs(w, seed=73, lengths=lengths)
+    _check(inp, O.llattn_quadratic(inp), "auto")
