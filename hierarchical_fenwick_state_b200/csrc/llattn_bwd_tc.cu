@@ -57,16 +57,19 @@ constexpr uint32_t kTileB = kC * 128;            // 128 rows x 128 B, 128-byte s
 constexpr uint32_t kOffQ = 0, kOffK = kTileB, kOffV = 2 * kTileB, kOffDO = 3 * kTileB;
 
 // Level kernel: a tile lies in one half of its block (half >= 128 tokens), so it needs two
-// inputs: X = K, Y = V on the left, X = Q, Y = dO on the right.  About 81 KB and 128 TMEM
-// columns, so two CTAs share an SM and overlap their tile chains.
+// inputs: X = K, Y = V on the left, X = Q, Y = dO on the right.  In pass 2 a whole tile's
+// gradient contributions are staged in the tiles the MMAs are done with (plus E) and added to
+// dq, dk, dv by TMA reduce-adds.  About 98 KB and 128 TMEM columns, so two CTAs share an SM
+// and overlap their tile chains.
 constexpr uint32_t kState = kD * 128;            // 64 rows x 128 B
-constexpr uint32_t kLOffX = 0, kLOffY = kTileB, kLOffXlo = 2 * kTileB;
-constexpr uint32_t kLOffShi = 3 * kTileB, kLOffSlo = kLOffShi + kState;
+constexpr uint32_t kLOffX = 0, kLOffY = kTileB, kLOffXlo = 2 * kTileB, kLOffE = 3 * kTileB;
+constexpr uint32_t kLOffShi = 4 * kTileB, kLOffSlo = kLOffShi + kState;
 constexpr uint32_t kLOffUhi = kLOffSlo + kState, kLOffUlo = kLOffUhi + kState;
 constexpr uint32_t kLOffDl = kLOffUlo + kState;  // dlam partials of column half 1: [128] fp32
 constexpr uint32_t kLOffBar = kLOffDl + kC * 4;  // [0] loads, [1] MMAs
 constexpr uint32_t kLOffMisc = kLOffBar + 16;    // [0] TMEM base, [1] abort
 constexpr uint32_t kSmemBytes = kLOffMisc + 16 + 1024;
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two level CTAs per SM");
 
 // ---- TMEM columns of the level kernel (128 allocated) ----
 constexpr uint32_t kColS = 0, kColU = 64;        // pass 1: M = 64 accumulators
@@ -102,7 +105,9 @@ __device__ __forceinline__ float2 bf2_at(const uint8_t* p) {
 __global__ void __launch_bounds__(kThreads, 2)
 bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-             const BwdProblem p, const double* __restrict__ g, int lvl) {
+             const __grid_constant__ CUtensorMap tdq, const __grid_constant__ CUtensorMap tdk,
+             const __grid_constant__ CUtensorMap tdv, const BwdProblem p,
+             const double* __restrict__ g, int lvl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -124,6 +129,7 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   uint8_t* tx = sm + kLOffX;
   uint8_t* ty = sm + kLOffY;
   uint8_t* txlo = sm + kLOffXlo;
+  uint8_t* te = sm + kLOffE;
   uint8_t* shi = sm + kLOffShi;
   uint8_t* slo = sm + kLOffSlo;
   uint8_t* uhi = sm + kLOffUhi;
@@ -145,6 +151,9 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
     prefetch_tensormap(&tmo);
+    prefetch_tensormap(&tdq);
+    prefetch_tensormap(&tdk);
+    prefetch_tensormap(&tdv);
   }
   tc_fence_before();
   __syncthreads();
@@ -299,10 +308,18 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   __syncthreads();
 
   // ---- pass 2: W = dO S^T (right tiles), DK = V U^T and DV = K U (left tiles) ----
+  // A whole tile's contributions go through shared memory to TMA reduce-adds (dq from Y and
+  // Xlo; dk from Y and Xlo, dv from X and E, one buffer per 32-column half): no gradient row is
+  // read into the SM, and the add happens in L2.  A tile running past the sequence end adds
+  // its rows by plain read-modify-writes instead.
   for (int j = 0; j < nt; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
     const bool left = t0 < mid;
+    const bool whole = t0 + kC <= sp.len;
+    // the previous tile's reduce-adds must have read their staging before X, Y are reloaded
+    if (tid == 0) bulk_wait_read();
+    if (!whole) __syncthreads();   // plain loads by every thread: after that wait
     const bool tma = load(t0, left);
     if (tma) bwait(0, ph_ld);
     tc_fence_before();
@@ -334,28 +351,28 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       }
       mma_commit(&bars[1]);
     }
-    // the gradient row this thread adds to is read while the MMAs run (dq on the right, dk on
-    // the left; dv after the first drain, to stay inside the register budget)
     const int t = t0 + row;
     const bool right_row = !left && t < rend;
     const bool left_row = left && t < lend;
     const size_t r = (right_row || left_row) ? row_of(t) : 0;
-    float* dst0 = (left ? p.dk : p.dq) + r * kD + 32 * hf;
-    float4 old0[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      old0[e] = (right_row || left_row) ? *reinterpret_cast<const float4*>(dst0 + 4 * e)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
     const double gt = (right_row || left_row) ? g[grow(t)] : gm;
     const float lam = right_row ? p.lam[r * p.L + lvl] : 0.f;
     bwait(1, ph_mma);
     tc_fence_after();
+    const bool ok = misc[1] == 0;
     float dlp = 0.f;
-    if (!left) {
+    if (whole) {
+      // staging of this thread's 32 columns of its row (128-byte swizzle, the reduce map's box)
+      auto stage = [&](uint8_t* dst, const float (&c)[32]) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + sw128_off(row, 2 * e)) =
+              make_float4(c[e], c[e + 1], c[e + 2], c[e + 3]);
+      };
       float w[32];
-      tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
-      tmem_wait_ld();
-      if (right_row && misc[1] == 0) {
+      if (!left) {
+        tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
+        tmem_wait_ld();
         const float sc = expf((float)(gt - gm));
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -363,34 +380,68 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
           const float2 q23 = bf2_at(tx + sw128_off(row, 32 * hf + e + 2));
           const float w0 = sc * w[e], w1 = sc * w[e + 1], w2 = sc * w[e + 2], w3 = sc * w[e + 3];
           dlp = fmaf(q01.x, w0, fmaf(q01.y, w1, fmaf(q23.x, w2, fmaf(q23.y, w3, dlp))));
-          float4 a = old0[e / 4];
+          w[e] = lam * w0;
+          w[e + 1] = lam * w1;
+          w[e + 2] = lam * w2;
+          w[e + 3] = lam * w3;
+        }
+        stage(hf ? txlo : ty, w);
+      } else {
+        const float f = expf((float)(gm - gt));
+        tmem_ld32(tmem + lane_off + kColDK + 32 * hf, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] *= f;
+        stage(hf ? txlo : ty, w);
+        tmem_ld32(tmem + lane_off + kColDV + 32 * hf, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] *= f;
+        stage(hf ? te : tx, w);
+      }
+      fence_proxy_async_smem();
+    } else if (!left) {
+      float w[32];
+      tmem_ld32(tmem + lane_off + kColW + 32 * hf, w);
+      tmem_wait_ld();
+      if (right_row && ok) {
+        float* dst = p.dq + r * kD + 32 * hf;
+        const float sc = expf((float)(gt - gm));
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float2 q01 = bf2_at(tx + sw128_off(row, 32 * hf + e));
+          const float2 q23 = bf2_at(tx + sw128_off(row, 32 * hf + e + 2));
+          const float w0 = sc * w[e], w1 = sc * w[e + 1], w2 = sc * w[e + 2], w3 = sc * w[e + 3];
+          dlp = fmaf(q01.x, w0, fmaf(q01.y, w1, fmaf(q23.x, w2, fmaf(q23.y, w3, dlp))));
+          float4 a = *reinterpret_cast<const float4*>(dst + e);
           a.x = fmaf(lam, w0, a.x);
           a.y = fmaf(lam, w1, a.y);
           a.z = fmaf(lam, w2, a.z);
           a.w = fmaf(lam, w3, a.w);
-          *reinterpret_cast<float4*>(dst0 + e) = a;
+          *reinterpret_cast<float4*>(dst + e) = a;
         }
       }
     } else {
-      const bool ok = left_row && misc[1] == 0;
-      const float f = ok ? expf((float)(gm - gt)) : 0.f;
+      const bool own = left_row && ok;
+      const float f = own ? expf((float)(gm - gt)) : 0.f;
       float v[32];
       tmem_ld32(tmem + lane_off + kColDK + 32 * hf, v);
       tmem_wait_ld();
-      if (ok) {
+      if (own) {
+        float* dk = p.dk + r * kD + 32 * hf;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          float4 a = old0[e / 4];
+          float4 a = *reinterpret_cast<float4*>(dk + e);
           a.x = fmaf(f, v[e], a.x);
           a.y = fmaf(f, v[e + 1], a.y);
           a.z = fmaf(f, v[e + 2], a.z);
           a.w = fmaf(f, v[e + 3], a.w);
-          *reinterpret_cast<float4*>(dst0 + e) = a;
+          *reinterpret_cast<float4*>(dk + e) = a;
         }
       }
       tmem_ld32(tmem + lane_off + kColDV + 32 * hf, v);
       tmem_wait_ld();
-      if (ok) {
+      if (own) {
         float* dv = p.dv + r * kD + 32 * hf;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -403,17 +454,28 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         }
       }
     }
-    if (!left) {
-      if (hf == 1) s_dl[row] = dlp;
-      __syncthreads();
-      if (hf == 0 && right_row && misc[1] == 0) p.dlam[row_of(t) * p.L + lvl] = dlp + s_dl[row];
-    }
+    if (!left && hf == 1) s_dl[row] = dlp;
     tc_fence_before();
-    __syncthreads();   // TMEM drained and the tiles free for the next one
+    __syncthreads();   // TMEM drained, the staging written, s_dl filled
+    if (!left && hf == 0 && right_row && ok) p.dlam[r * p.L + lvl] = dlp + s_dl[row];
+    if (whole && tid == 0 && misc[1] == 0) {
+      const int z = (int)(sp.start + t0);
+      if (!left) {
+        tma_reduce_add_3d(&tdq, ty, 0, h, z);
+        tma_reduce_add_3d(&tdq, txlo, 32, h, z);
+      } else {
+        tma_reduce_add_3d(&tdk, ty, 0, h, z);
+        tma_reduce_add_3d(&tdk, txlo, 32, h, z);
+        tma_reduce_add_3d(&tdv, tx, 0, h, z);
+        tma_reduce_add_3d(&tdv, te, 32, h, z);
+      }
+      bulk_commit();
+    }
   }
 
   // a copy or MMA batch whose wait timed out must land before the CTA exits
   if (stuck >= 0 && tid == 0) mbar_wait(&bars[stuck], stuck_par, 100000000ull);
+  if (tid == 0) bulk_wait_all();   // the reduce-adds have read their staging and landed
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -708,12 +770,15 @@ cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st)
   // TMA only fetches whole tiles inside a sequence, so for a packed batch any token extent
   // >= the real total serves (nseq * T bounds it)
   const long long tokens = (long long)p.nseq * p.T;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mdq, mdk, mdv;
   cudaError_t e;
   if ((e = make_map(&mq, p.q, kD, p.H, tokens)) != cudaSuccess ||
       (e = make_map(&mk, p.k, kD, p.H, tokens)) != cudaSuccess ||
       (e = make_map(&mv, p.v, kD, p.H, tokens)) != cudaSuccess ||
-      (e = make_map(&mo, p.dout, kD, p.H, tokens)) != cudaSuccess)
+      (e = make_map(&mo, p.dout, kD, p.H, tokens)) != cudaSuccess ||
+      (e = make_out_map(&mdq, p.dq, kD, p.H, tokens)) != cudaSuccess ||
+      (e = make_out_map(&mdk, p.dk, kD, p.H, tokens)) != cudaSuccess ||
+      (e = make_out_map(&mdv, p.dv, kD, p.H, tokens)) != cudaSuccess)
     return e;
   static std::atomic<bool> attr_set[64];
   int dev = 0;
@@ -732,7 +797,8 @@ cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st)
   count_launch();
   for (int lvl = kTcFirstLevel; lvl < p.L; ++lvl) {
     const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
-    bwd_level_tc<<<dim3(nblk, p.H, p.nseq), kThreads, kSmemBytes, st>>>(mq, mk, mv, mo, p, g, lvl);
+    bwd_level_tc<<<dim3(nblk, p.H, p.nseq), kThreads, kSmemBytes, st>>>(mq, mk, mv, mo, mdq, mdk, mdv,
+                                                                         p, g, lvl);
     count_launch();
   }
   return cudaGetLastError();

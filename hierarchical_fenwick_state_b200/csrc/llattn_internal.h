@@ -49,6 +49,10 @@ bool tc_serial_supports(int in_dtype, int dk, int dv, int chunk, int T);
 // TMA map of a [tokens, H, rowlen] bf16 tensor viewed as {rowlen, H, tokens}: box {64, 1, 128}
 // (one 64-column slice of 128 rows), 128-byte swizzle.
 cudaError_t make_map(CUtensorMap* m, const void* base, int rowlen, int H, long long tokens);
+// TMA map of a [tokens, H, rowlen] fp32 tensor viewed as {rowlen, H, tokens}: box {32, 1, 128}
+// (one 32-column slice of 128 rows, 128-byte rows), 128-byte swizzle; for tile stores and
+// reduce-adds.
+cudaError_t make_out_map(CUtensorMap* m, void* base, int rowlen, int H, long long tokens);
 
 // Device address of the fixed scratch array behind llattn_fwd_noalloc on the
 // current device (looked up on the first call per device, then cached).

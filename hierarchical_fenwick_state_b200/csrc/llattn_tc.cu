@@ -1615,8 +1615,6 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int rowlen, int H, long l
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-namespace {
-
 // out [tokens, H, rowlen] fp32 as {rowlen, H, tokens}; box {32, 1, 128} (128 B rows), 128 B swizzle.
 cudaError_t make_out_map(CUtensorMap* m, void* base, int rowlen, int H, long long tokens) {
   EncodeTiledFn enc = encode_fn();
@@ -1630,6 +1628,8 @@ cudaError_t make_out_map(CUtensorMap* m, void* base, int rowlen, int H, long lon
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+namespace {
 
 int sm_count() {
   int dev = 0, n = 0;
