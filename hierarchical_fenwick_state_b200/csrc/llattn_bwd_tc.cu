@@ -107,13 +107,18 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
              const __grid_constant__ CUtensorMap tdq, const __grid_constant__ CUtensorMap tdk,
              const __grid_constant__ CUtensorMap tdv, const BwdProblem p,
-             const double* __restrict__ g, int lvl) {
+             const double* __restrict__ g, int lvl, int split) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = warp & 3, hf = warp >> 2, row = sub * 32 + lane;
   const uint32_t lane_off = uint32_t(sub * 32) << 16;
-  const int blk = blockIdx.x, h = blockIdx.y, sq = blockIdx.z;
+  // split != 0: two CTAs per block, blockIdx.x = 2 * block + side.  The key side (0) reduces U
+  // over the right half and adds into dk, dv of the left; the query side (1) reduces S over the
+  // left half and adds into dq, dlam of the right.  Otherwise one CTA does both.
+  const int blk = split ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int side = split ? (int)(blockIdx.x & 1) : -1;
+  const int h = blockIdx.y, sq = blockIdx.z;
   const SeqSpan sp = seq_span(sq, p.T, p.cu_seqlens, p.status);
   const int half = 1 << (lvl - 1);               // a multiple of 128 (lvl >= 8)
   const long long a0 = (long long)blk << lvl;
@@ -123,7 +128,8 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   const int rend = (int)min((long long)lo + 2 * half, (long long)sp.len);    // right [mid, rend)
   auto row_of = [&](int t) { return (size_t)(sp.start + t) * p.H + h; };
   auto grow = [&](int t) { return ((size_t)sq * p.T + t) * p.H + h; };
-  for (int t = lo + tid; t < lend; t += kThreads) p.dlam[row_of(t) * p.L + lvl] = 0.f;
+  if (side <= 0)
+    for (int t = lo + tid; t < lend; t += kThreads) p.dlam[row_of(t) * p.L + lvl] = 0.f;
   if (mid >= sp.len) return;   // no right half: nothing meets at this level
 
   uint8_t* tx = sm + kLOffX;
@@ -209,6 +215,11 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   const uint32_t xa = smem_u32(tx), ya = smem_u32(ty), xla = smem_u32(txlo);
   const uint32_t sha = smem_u32(shi), sla = smem_u32(slo), uha = smem_u32(uhi), ula = smem_u32(ulo);
   const int nt = (rend - lo + kC - 1) / kC;
+  const int nl = (lend - lo + kC - 1) / kC;   // tiles [0, nl) are left, [nl, nt) right
+  // the tiles each pass walks: both halves, or for a split block the other side's half in
+  // pass 1 and this side's half in pass 2
+  const int p1b = side == 0 ? nl : 0, p1e = side == 1 ? nl : nt;
+  const int p2b = side == 1 ? nl : 0, p2e = side == 0 ? nl : nt;
 
   // ---- pass 1: S = sum exp(g_m - g_s) k_s v_s^T (left), U = sum lam exp(g_t - g_m) q_t do_t^T ----
   bool s_started = false, u_started = false;
@@ -225,8 +236,8 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   };
   double g_next;
   float l_next;
-  row_in(0, g_next, l_next);
-  for (int j = 0; j < nt; ++j) {
+  row_in(p1b, g_next, l_next);
+  for (int j = p1b; j < p1e; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
     const bool left = t0 < mid;
@@ -312,7 +323,7 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   // Xlo; dk from Y and Xlo, dv from X and E, one buffer per 32-column half): no gradient row is
   // read into the SM, and the add happens in L2.  A tile running past the sequence end adds
   // its rows by plain read-modify-writes instead.
-  for (int j = 0; j < nt; ++j) {
+  for (int j = p2b; j < p2e; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
     const bool left = t0 < mid;
@@ -759,6 +770,16 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   }
 }
 
+constexpr int kSplitDen = 2;   // split a level whose blocks fill at most 1 / kSplitDen of the slots
+
+int sm_count_bwd() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
 }  // namespace
 
 bool bwd_tc_supports(const BwdProblem& p) {
@@ -795,10 +816,13 @@ cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st)
   // levels 0..7: one CTA per chunk, the first write of dq, dk, dv and dlam[:, 0..7]
   bwd_intra_tc<<<dim3((p.T + kC - 1) / kC, p.H, p.nseq), kThreads, kISmemBytes, st>>>(mq, mk, mv, mo, p, g);
   count_launch();
+  const long long slots = 2ll * sm_count_bwd();   // two level CTAs per SM
   for (int lvl = kTcFirstLevel; lvl < p.L; ++lvl) {
     const int nblk = (int)(((long long)p.T + (1ll << lvl) - 1) >> lvl);
-    bwd_level_tc<<<dim3(nblk, p.H, p.nseq), kThreads, kSmemBytes, st>>>(mq, mk, mv, mo, mdq, mdk, mdv,
-                                                                         p, g, lvl);
+    // blocks that leave CTA slots free are taken by two CTAs each (half the tile steps each)
+    const int split = (long long)nblk * p.H * p.nseq * kSplitDen <= slots ? 1 : 0;
+    bwd_level_tc<<<dim3(nblk << split, p.H, p.nseq), kThreads, kSmemBytes, st>>>(
+        mq, mk, mv, mo, mdq, mdk, mdv, p, g, lvl, split);
     count_launch();
   }
   return cudaGetLastError();
