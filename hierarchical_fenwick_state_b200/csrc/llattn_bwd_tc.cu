@@ -17,7 +17,12 @@
 // over the tiles on the tensor cores (K^T V and Q^T dO shapes, M = 64, the token index as the
 // reduction dimension) into TMEM.  Pass 2 multiplies every tile by them: W = dO S^T,
 // DK = V U^T, DV = K U (M = 128 rows per tile), and the epilogue applies the exponential
-// factors, forms dlam and adds into dq, dk, dv.
+// factors, forms dlam and adds into dq, dk, dv: a whole tile's contributions are staged in
+// shared memory and added by TMA reduce-adds (the add happens in L2, no gradient row is read
+// into the SM); a tile that runs past the sequence end adds its rows by plain
+// read-modify-writes.  A level whose blocks fill at most half the CTA slots (two per SM) runs
+// two CTAs per block: the key side reduces U and adds into the left half's dk, dv, the query
+// side reduces S and adds into the right half's dq, dlam.
 //
 // Precision: q, k, v and dO enter as the bf16 values they are.  The operands the method derives
 // (the decay-scaled rows of K and Q, and S, U) are split into a bf16 high part and a bf16
