@@ -532,7 +532,9 @@ __device__ __forceinline__ uint64_t mndesc2(uint32_t saddr) { return sdesc_sw128
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-             const BwdProblem p, const double* __restrict__ g) {
+             const __grid_constant__ CUtensorMap tdq, const __grid_constant__ CUtensorMap tdk,
+             const __grid_constant__ CUtensorMap tdv, const BwdProblem p,
+             const double* __restrict__ g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -749,20 +751,44 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   bwait(1, ph_mma);
   ph_mma ^= 1u;
   tc_fence_after();
+  // A whole chunk's dq, dk, dv go through the spent P tiles (one 16 KB half per 32 columns, in
+  // the 128-byte swizzle of the store map's box) to TMA tile stores: whole 128-byte rows, where
+  // per-thread row stores would touch 32 lines per warp instruction.  A ragged last chunk
+  // stores its rows with plain stores (a whole box would reach the next sequence's rows).
   {
     const bool ok = row < n && misc[1] == 0;
     const size_t r = ok ? row_of(t0 + row) * kD + 32 * hf : 0;
-    const struct { uint32_t col; float* dst; } outs[3] = {
-        {kIColDQ, p.dq}, {kIColDK, p.dk}, {kIColDV, p.dv}};
+    const struct { uint32_t col; float* dst; uint8_t* stage; const CUtensorMap* map; } outs[3] = {
+        {kIColDQ, p.dq, p1h, &tdq}, {kIColDK, p.dk, p1l, &tdk}, {kIColDV, p.dv, p2h, &tdv}};
 #pragma unroll
     for (int x = 0; x < 3; ++x) {
       float v[32];
       tmem_ld32(tmem + lane_off + outs[x].col + 32 * hf, v);
       tmem_wait_ld();
-      if (ok) {
+      if (tma) {
+        uint8_t* dst = outs[x].stage + hf * kHalfB;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + sw128_off(row, 2 * e)) =
+              make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      } else if (ok) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
           *reinterpret_cast<float4*>(outs[x].dst + r + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      }
+    }
+    if (tma) {
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0 && misc[1] == 0) {
+        const int z = (int)(sp.start + t0);
+#pragma unroll
+        for (int x = 0; x < 3; ++x) {
+          tma_store_3d(outs[x].map, outs[x].stage, 0, h, z);
+          tma_store_3d(outs[x].map, outs[x].stage + kHalfB, 32, h, z);
+        }
+        bulk_commit();
+        bulk_wait_all();   // the stores have read the staging and landed before the CTA exits
       }
     }
   }
@@ -819,7 +845,8 @@ cudaError_t bwd_levels_tc(const BwdProblem& p, const double* g, cudaStream_t st)
     attr_set[dev].store(true);
   }
   // levels 0..7: one CTA per chunk, the first write of dq, dk, dv and dlam[:, 0..7]
-  bwd_intra_tc<<<dim3((p.T + kC - 1) / kC, p.H, p.nseq), kThreads, kISmemBytes, st>>>(mq, mk, mv, mo, p, g);
+  bwd_intra_tc<<<dim3((p.T + kC - 1) / kC, p.H, p.nseq), kThreads, kISmemBytes, st>>>(
+      mq, mk, mv, mo, mdq, mdk, mdv, p, g);
   count_launch();
   const long long slots = 2ll * sm_count_bwd();   // two level CTAs per SM
   for (int lvl = kTcFirstLevel; lvl < p.L; ++lvl) {
