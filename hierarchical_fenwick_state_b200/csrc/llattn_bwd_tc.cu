@@ -328,6 +328,20 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   // Xlo; dk from Y and Xlo, dv from X and E, one buffer per 32-column half): no gradient row is
   // read into the SM, and the add happens in L2.  A tile running past the sequence end adds
   // its rows by plain read-modify-writes instead.
+  // this row's prefix sum (and lam on the right) of pass-2 tile j, read one tile ahead
+  auto row2_in = [&](int j, double& gt, float& lt) {
+    const int t = lo + j * kC + row;
+    const bool left = lo + j * kC < mid;
+    gt = gm;
+    lt = 0.f;
+    if (j < p2e && t < (left ? lend : rend)) {
+      gt = g[grow(t)];
+      if (!left) lt = p.lam[row_of(t) * p.L + lvl];
+    }
+  };
+  double g2_next;
+  float l2_next;
+  row2_in(p2b, g2_next, l2_next);
   for (int j = p2b; j < p2e; ++j) {
     if (misc[1] != 0) break;
     const int t0 = lo + j * kC;
@@ -371,8 +385,9 @@ bwd_level_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     const bool right_row = !left && t < rend;
     const bool left_row = left && t < lend;
     const size_t r = (right_row || left_row) ? row_of(t) : 0;
-    const double gt = (right_row || left_row) ? g[grow(t)] : gm;
-    const float lam = right_row ? p.lam[r * p.L + lvl] : 0.f;
+    const double gt = g2_next;
+    const float lam = l2_next;
+    row2_in(j + 1, g2_next, l2_next);
     bwait(1, ph_mma);
     tc_fence_after();
     const bool ok = misc[1] == 0;
