@@ -41,6 +41,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <type_traits>
 
 #include "../../include/llattn.h"
 #include "llattn_bwd.h"
@@ -532,7 +533,8 @@ constexpr uint32_t kIOffP2h = kIOffP1l + kMatB, kIOffP2l = kIOffP2h + kMatB;
 constexpr uint32_t kIOffG = kIOffP2l + kMatB;         // g of the chunk's rows: [128] fp64
 constexpr uint32_t kIOffLam = kIOffG + kC * 8;        // lam[t, 0..7]: [128][9] fp32 (odd stride)
 constexpr uint32_t kIOffDl = kIOffLam + kC * 9 * 4;   // dlam partials of column half 1: [128][8]
-constexpr uint32_t kIOffBar = kIOffDl + kC * 8 * 4;
+constexpr uint32_t kIOffCj = kIOffDl + kC * 8 * 4;   // exp(g_0 - g_s) of the chunk's keys: [128]
+constexpr uint32_t kIOffBar = kIOffCj + kC * 4;
 constexpr uint32_t kIOffMisc = kIOffBar + 16;
 constexpr uint32_t kISmemBytes = kIOffMisc + 16 + 1024;
 static_assert(kISmemBytes <= 227 * 1024, "shared memory");
@@ -573,6 +575,7 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   double* s_g = reinterpret_cast<double*>(sm + kIOffG);
   float* s_lam = reinterpret_cast<float*>(sm + kIOffLam);
   float* s_dl = reinterpret_cast<float*>(sm + kIOffDl);
+  float* s_cj = reinterpret_cast<float*>(sm + kIOffCj);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kIOffBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kIOffMisc);
 
@@ -623,6 +626,12 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Decay of a pair: exp(g_t - g_s) = exp(g_t - g_0) exp(g_0 - g_s) when the chunk's decay
+  // range is at most 80, where both factors are normal fp32 numbers (one product per pair, the
+  // key factors tabled once); a chunk of stronger decay takes exp(g_t - g_s) pair by pair.
+  const double g0 = s_g[0];
+  const bool factored = g0 - s_g[n - 1] <= 80.0;
+  if (hf == 1) s_cj[row] = (factored && row < n) ? expf((float)(g0 - s_g[row])) : 0.f;
   const uint32_t tmem = misc[0];
   uint32_t ph_mma = 0u;
   int stuck = -1;
@@ -658,6 +667,7 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   tc_fence_after();
 
   // ---- masks: P1 = M .* B, P2 = M .* A (hi / lo), and dlam's level sums ----
+  __syncthreads();   // the key factors are in place
   {
     const int t = row;
     const double gt = s_g[t];
@@ -666,6 +676,11 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
 #pragma unroll
     for (int l = 0; l < 8; ++l) dl[l] = 0.f;
     const uint32_t hoff = hf * kHalfB;   // this thread's columns are half hf of each matrix
+    const float rsc = (factored && t < n) ? expf((float)(gt - g0)) : 0.f;
+    auto masks = [&](auto fac) {
+    constexpr bool kFac = decltype(fac)::value;
+    // decay of the pair (t, s)
+    auto decay = [&](int s) { return kFac ? rsc * s_cj[s] : expf((float)(gt - s_g[s])); };
 #pragma unroll 1
     for (int c16 = 0; c16 < 4; ++c16) {
       const int s0 = 64 * hf + 16 * c16;
@@ -685,7 +700,7 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
             float xs = 0.f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float E = expf((float)(gt - s_g[s0 + e]));
+              const float E = decay(s0 + e);
               const float m = lam * E;
               p1[e] = m * bv[e];
               p2[e] = m * av[e];
@@ -699,7 +714,7 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
             for (int e = 0; e < 16; ++e) {
               const int s = s0 + e;
               if (s <= t) {
-                const float E = expf((float)(gt - s_g[s]));
+                const float E = decay(s);
                 const int lev = 32 - __clz(t ^ s);   // 0 when s == t
                 const float m = lr[lev] * E;
                 p1[e] = m * bv[e];
@@ -727,6 +742,9 @@ bwd_intra_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         *reinterpret_cast<uint4*>(p2l + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
       }
     }
+    };
+    if (factored) masks(std::true_type{});
+    else masks(std::false_type{});
     if (hf == 1) {
 #pragma unroll
       for (int l = 0; l < 8; ++l) s_dl[t * 8 + l] = dl[l];
