@@ -403,3 +403,43 @@ def test_short_sequences_packed_cluster_split():
     w = I.Workload("short_vl4", B=len(lengths), H=2, T=128, dk=64, dv=64, dtype="f32", varlen=True)
     inp = I.make_inputs(w, seed=73, lengths=lengths)
     _check(inp, O.llattn_quadratic(inp), "auto")
+
+
+# ------------------------------------------------------------------------------------------------
+# A call captured in a CUDA graph (how the benchmark issues its steps) computes what the direct
+# call computes
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name,B,H,T,dtype,dk,segments", [
+    ("segmented", 2, 4, 2048, "bf16", 64, True),    # pre-pass kernels and dependent launches
+    ("whole", 4, 32, 700, "bf16", 64, False),       # one CTA per (sequence, head)
+    ("short", 2, 4, 300, "f32", 32, None),          # the one-launch masked form
+])
+def test_graph_replay_matches_direct_call(name, B, H, T, dtype, dk, segments):
+    import torch
+    w = I.Workload("graph_" + name, B=B, H=H, T=T, dk=dk, dv=dk, dtype=dtype)
+    inp = I.make_inputs(w, seed=T + dk)
+    t = _to_device_for_guard(inp)
+    args = (t["q"], t["k"], t["v"], t["log_a"], t["lam"])
+    direct = binding.forward(*args)
+    torch.cuda.synchronize()
+    if segments is not None:
+        cut = binding.segment_plan(inp.B, inp.H, inp.T, inp.dk, inp.dv, False) > 0
+        assert cut == segments
+    out = torch.full_like(direct, float("nan"))
+    ws = torch.empty(max(binding.workspace_bytes(1 if dtype == "bf16" else 0, "auto", 0, inp.B,
+                                                 inp.H, inp.T, inp.dk, inp.dv, False), 256),
+                     dtype=torch.uint8, device="cuda:0")
+    binding.forward(*args, out=out, workspace=ws)          # first call outside the capture
+    torch.cuda.synchronize()
+    out.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        binding.forward(*args, out=out, workspace=ws)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert binding.stream_status(clear=True) == 0
+    assert torch.equal(out, direct), "a replayed call differs from the direct call"
+    err = O.rel_max_err(out.double().cpu().numpy(), O.llattn_recurrent(inp))
+    assert err <= TOL[inp.dtype], f"rel max err {err:.3e}"
+    del g
