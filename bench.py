@@ -975,6 +975,20 @@ def run_bwd(args, w, rank, world, local_rank):
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
+    # as for the forward: the call captured once as a CUDA graph and replayed (--graph off:
+    # every call issued from Python)
+    use_graph = args.graph != "off"
+    graph = None
+    if use_graph:
+        binding.profile_read(reset=True)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        launches_per_step = binding.profile_read(reset=True)[2]
+        for _ in range(max(args.warmup, 3)):
+            graph.replay()
+        torch.cuda.synchronize()
     binding.profile_read(reset=True)
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -986,7 +1000,10 @@ def run_bwd(args, w, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
     e1.record(stream)
     torch.cuda.synchronize()
     if dist:
@@ -995,6 +1012,9 @@ def run_bwd(args, w, rank, world, local_rank):
     clk = clocks.stop()
     ms_total = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     main_ms, main_n, launches = binding.profile_read(reset=True)
+    if graph is not None:
+        launches, main_n = launches_per_step * args.steps, 0   # the step's time is the call's
+        del graph
     status = binding.device_status(clear=True)
     if status:
         raise RuntimeError(f"device status flags {status:#x} after the timed region")
@@ -1035,8 +1055,9 @@ def run_bwd(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": bwd_config(w, "tensor cores: chunk pairs, then level by level" if tensor
-                             else "simt level-by-level"),
+        "config": {**bwd_config(w, "tensor cores: chunk pairs, then level by level" if tensor
+                                else "simt level-by-level"),
+                   **({"launch": "CUDA graph of one step, replayed"} if use_graph else {})},
         "roofline": roof, "gpu_launches": launches, "clocks": clk,
     }
 

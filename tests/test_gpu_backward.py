@@ -136,3 +136,39 @@ def test_backward_at_the_benchmark_size_sampled():
         mine = got["log_a"].reshape(total, inp.H)[sl, h]
         err = O.rel_max_err(mine, dref)
         assert err <= TOL, f"dlog_a (sequence {b}, head {h}): rel max err {err:.3e}"
+
+
+def test_backward_graph_replay_matches_direct_call():
+    """The backward captured in a CUDA graph (how the benchmark issues its steps) writes the
+    same gradients as the direct call, bit for bit."""
+    import torch
+    w = I.shrink(W["t2k_d64_bf16"], B=2, H=2, T=1500)
+    inp = I.make_inputs(w, seed=33)
+    do = _do(inp, 34)
+    direct = _run(inp, do)
+    tdt = torch.bfloat16
+    dev = torch.device("cuda:0")
+    t = {n: torch.from_numpy(getattr(inp, n)).to(dev) for n in NAMES}
+    for n in ("q", "k", "v"):
+        t[n] = t[n].to(tdt)
+    tdo = torch.from_numpy(do.astype(np.float32)).to(dev).to(tdt)
+    grads = {n: torch.full(getattr(inp, n).shape, float("nan"), dtype=torch.float32, device=dev)
+             for n in NAMES}
+    ws = torch.empty(max(binding.bwd_workspace_bytes(inp.B, inp.H, inp.T, inp.dk, inp.dv), 256),
+                     dtype=torch.uint8, device=dev)
+    call = lambda: binding.backward(t["q"], t["k"], t["v"], t["log_a"], t["lam"], tdo, T=inp.T,
+                                    grads=grads, workspace=ws)
+    call()                                   # first call outside the capture
+    torch.cuda.synchronize()
+    for g_ in grads.values():
+        g_.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert binding.device_status(clear=True) == 0
+    for n in NAMES:
+        assert np.array_equal(grads[n].double().cpu().numpy(), direct[n]), f"d{n} differs after replay"
+    del g
