@@ -513,13 +513,15 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     # The step is captured once as a CUDA graph after the warm-up calls and replayed: the same
     # kernels on the same resident inputs, without the per-call host cost (argument checks and
-    # marshalling in Python, the driver's launches), which bounds short steps.
+    # marshalling in Python, the driver's launches), which bounds short steps.  The capture
+    # checks only this thread's calls: under torchrun the process group's own threads may query
+    # events meanwhile.
     use_graph = args.graph != "off"
     graph = None
     if use_graph:
         binding.profile_read(reset=True)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             step()
         torch.cuda.synchronize()
         launches_per_step = binding.profile_read(reset=True)[2]
@@ -982,7 +984,7 @@ def run_bwd(args, w, rank, world, local_rank):
     if use_graph:
         binding.profile_read(reset=True)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             step()
         torch.cuda.synchronize()
         launches_per_step = binding.profile_read(reset=True)[2]
